@@ -1,0 +1,27 @@
+"""Build the CPU oracle (oracle.c -> liboracle.so) with gcc.
+
+Test infrastructure: the product library never links this.  Compiled with
+-O2 and without -ffast-math so that fp64 arithmetic follows IEEE order.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= max(
+        os.path.getmtime(SRC), os.path.getmtime(os.path.join(HERE, "oracle.h"))
+    ):
+        return LIB
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+           "-fno-fast-math", "-Wall", "-Wextra", "-o", LIB, SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))
