@@ -1,0 +1,135 @@
+"""Python binding of libqmv, the B200 (sm_100a) affine group-quantized GEMV.
+
+Argument marshalling only: every function here forwards to the C entry point
+of the same name in ``libqmv.so`` (declared in ``include/qmv.h``) and every
+step of the computation runs in that library's CUDA kernels.  There is no
+CPU path: if ``libqmv.so`` is missing or no CUDA device is usable, calls
+raise.
+
+Arguments may be ``torch.Tensor`` (CUDA, contiguous; the data pointer is
+passed) or plain integer device addresses.  bf16 buffers are ``torch.bfloat16``
+tensors (or any 2-byte dtype holding bf16 bit patterns), packed weights are
+``torch.int32``/``torch.uint32`` tensors.  ``stream`` defaults to the current
+torch CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmv.so")
+
+QMV_OK = 0
+QMV_ERR_NULL = 1
+QMV_ERR_SHAPE = 2
+QMV_ERR_UNSUPPORTED = 3
+QMV_ERR_ALIGN = 4
+QMV_ERR_CUDA = 5
+
+_STATUS_NAMES = {0: "QMV_OK", 1: "QMV_ERR_NULL", 2: "QMV_ERR_SHAPE",
+                 3: "QMV_ERR_UNSUPPORTED", 4: "QMV_ERR_ALIGN", 5: "QMV_ERR_CUDA"}
+
+
+class QmvError(RuntimeError):
+    """A libqmv entry point returned a nonzero status."""
+
+    def __init__(self, func: str, status: int, message: str):
+        self.status = status
+        super().__init__(f"{func}: {_STATUS_NAMES.get(status, status)}: {message}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqmv.so (built in-tree by ``affine_group_quantized_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m affine_group_quantized_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.qmv.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+        L.qmv_gate_up.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P]
+        L.qmv_silu_gate_resid.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
+        L.gather_qmv.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                 P, P]
+        for f in (L.qmv, L.qmv_gate_up, L.qmv_silu_gate_resid, L.gather_qmv):
+            f.restype = I
+        L.qmv_last_error.restype = ctypes.c_char_p
+        L.qmv_last_error.argtypes = []
+        L.qmv_abi_version.restype = I
+        L.qmv_abi_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("qmv", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
+            "qmv_last_error", "qmv_abi_version")
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(func: str, rc: int):
+    if rc != QMV_OK:
+        raise QmvError(func, rc, lib().qmv_last_error().decode())
+
+
+def last_error() -> str:
+    return lib().qmv_last_error().decode()
+
+
+def abi_version() -> int:
+    return lib().qmv_abi_version()
+
+
+def qmv(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):
+    """y[M,N] = x[M,K] @ dequant(w).T  (see include/qmv.h)."""
+    _check("qmv", lib().qmv(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases),
+                            _ptr(y), M, N, K, bits, group_size, _stream(stream)))
+
+
+def qmv_gate_up(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up,
+                M, N, K, bits, group_size, stream=None):
+    """y_gate = x @ dequant(w_gate).T and y_up = x @ dequant(w_up).T, one launch."""
+    _check("qmv_gate_up", lib().qmv_gate_up(
+        _ptr(x), _ptr(w_gate), _ptr(s_gate), _ptr(b_gate), _ptr(w_up),
+        _ptr(s_up), _ptr(b_up), _ptr(y_gate), _ptr(y_up), M, N, K, bits,
+        group_size, _stream(stream)))
+
+
+def qmv_silu_gate_resid(gate, up, x_resid, w, scales, biases, y, M, N, K,
+                        bits, group_size, stream=None):
+    """y = x_resid + dequant(w) @ (silu(gate) * up); x_resid may be None."""
+    _check("qmv_silu_gate_resid", lib().qmv_silu_gate_resid(
+        _ptr(gate), _ptr(up), _ptr(x_resid), _ptr(w), _ptr(scales),
+        _ptr(biases), _ptr(y), M, N, K, bits, group_size, _stream(stream)))
+
+
+def gather_qmv(x, w, scales, biases, lhs_indices, rhs_indices, y, num_pairs,
+               num_x_rows, num_experts, N, K, bits, group_size,
+               sorted_indices=False, d_status=None, stream=None):
+    """y[p] = x[lhs[p]] @ dequant(w[rhs[p]]).T for every pair p."""
+    _check("gather_qmv", lib().gather_qmv(
+        _ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(lhs_indices),
+        _ptr(rhs_indices), _ptr(y), num_pairs, num_x_rows, num_experts, N, K,
+        bits, group_size, 1 if sorted_indices else 0, _ptr(d_status),
+        _stream(stream)))

@@ -1,0 +1,404 @@
+// qmv_api.cu -- the C ABI of libqmv: argument checks, launch planning and
+// kernel dispatch.  Declarations and the contract of every entry point are in
+// include/qmv.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "qmv.h"
+#include "qmv_stream.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return QMV_OK;
+}
+
+bool aligned16(const void *p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool bits_supported(int bits) {
+  return bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 ||
+         bits == 8;
+}
+
+bool gs_supported(int gs) { return gs == 32 || gs == 64 || gs == 128; }
+
+int gcd_i(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+// Per-device facts, queried once per device.
+struct DeviceInfo {
+  int sms = 0;
+  int smem_optin = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+int device_info(DeviceInfo **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return fail(QMV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(QMV_ERR_CUDA, "device index %d out of range", dev);
+  int rc = QMV_OK;
+  std::call_once(g_dev_once[dev], [&] {
+    cudaError_t e1 = cudaDeviceGetAttribute(&g_dev[dev].sms,
+                                            cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e2 = cudaDeviceGetAttribute(
+        &g_dev[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e1 != cudaSuccess || e2 != cudaSuccess) g_dev[dev].sms = 0;
+  });
+  if (g_dev[dev].sms <= 0)
+    return fail(QMV_ERR_CUDA, "cannot query device %d attributes", dev);
+  *out = &g_dev[dev];
+  return rc;
+}
+
+// Common shape checks of the pages' shape rule: w holds K*bits/32 words per
+// row and K/group_size groups (extract_quantized_matmul_dims).
+int check_common(int N, int K, int bits, int gs) {
+  if (!bits_supported(bits))
+    return fail(QMV_ERR_UNSUPPORTED, "bits=%d not in {2,3,4,5,6,8}", bits);
+  if (!gs_supported(gs))
+    return fail(QMV_ERR_UNSUPPORTED, "group_size=%d not in {32,64,128}", gs);
+  if (N <= 0) return fail(QMV_ERR_SHAPE, "N=%d must be positive", N);
+  if (K <= 0) return fail(QMV_ERR_SHAPE, "K=%d must be positive", K);
+  if (K % gs != 0)
+    return fail(QMV_ERR_SHAPE, "K=%d is not a multiple of group_size=%d", K, gs);
+  if (K > 28672)
+    return fail(QMV_ERR_UNSUPPORTED, "K=%d above the supported 28672", K);
+  return QMV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Launch planning for the streaming kernel
+// ---------------------------------------------------------------------------
+struct Plan {
+  qmvk::StreamParams p;
+  int mr = 1, nsl = 1;
+  int threads = 0;
+  size_t smem = 0;
+  int grid = 0;
+};
+
+int make_plan(Plan &pl, int bits, int gs, int mr_want, long long work_rows,
+              DeviceInfo *dev) {
+  qmvk::StreamParams &p = pl.p;
+  const int K = p.K;
+  const int U = K / 32;
+  int Upad, nsl = 1, PH = 1;
+  if (U >= 32) {
+    Upad = (U + 31) / 32 * 32;
+  } else {
+    Upad = 1;
+    while (Upad < U) Upad <<= 1;
+  }
+  if (Upad > 448) {
+    Upad = (U + 63) / 64 * 64;
+    nsl = 2;
+  } else {
+    PH = Upad <= 256 ? (256 + Upad - 1) / Upad : 1;
+  }
+  const int Tc = Upad * PH / nsl;
+  if (Tc > 448 || Tc % 32 != 0)
+    return fail(QMV_ERR_UNSUPPORTED, "K=%d has no thread layout", K);
+  const int L = Upad < 32 ? Upad : 32;
+  const int mr = (nsl == 1 && mr_want >= 2 && L >= 2) ? 2 : 1;
+  const long long row_bytes = static_cast<long long>(K) * bits / 8;
+  const int G = K / gs;
+  // rows per thread per tile: largest power of two with RPT*MR <= L that
+  // keeps one stage's weight bytes within 32 KB
+  int RPT = 8;
+  while (RPT > 1 && (RPT * mr > L || static_cast<long long>(RPT) * PH * row_bytes > 32768))
+    RPT >>= 1;
+  const int RT = RPT * PH;
+  const int ra_w = 16 / gcd_i(static_cast<int>(row_bytes % 16 == 0 ? 16 : row_bytes % 16), 16);
+  const int ra_s = 16 / gcd_i((2 * G) % 16 == 0 ? 16 : (2 * G) % 16, 16);
+  const int RA = ra_w * ra_s / gcd_i(ra_w, ra_s);
+  const long long stage_rows = RT + RA - 1;
+  const long long w_stage = (stage_rows * row_bytes + 15 + 15) / 16 * 16;
+  const long long s_stage = (stage_rows * 2LL * G + 15 + 15) / 16 * 16;
+  const long long stage_bytes = w_stage + 2 * s_stage;
+  const int wpr = Upad >= 32 ? Upad / 32 / nsl : 1;
+  const long long red_bytes = 2LL * RT * mr * wpr * 4;
+  long long grp_bytes = 0;
+  if (p.mode == qmvk::MODE_GATHER)
+    grp_bytes = (3LL * p.num_experts + 1 + p.num_pairs) * 4;
+  const long long budget = dev->smem_optin;
+  const long long fixed = 2LL * 8 * 8 + red_bytes + grp_bytes + 256;
+  long long ns = (budget - fixed) / stage_bytes;
+  if (ns > 8) ns = 8;
+  if (ns < 2)
+    return fail(QMV_ERR_UNSUPPORTED,
+                "shape needs more shared memory than the device offers "
+                "(stage %lld B, fixed %lld B)",
+                stage_bytes, fixed);
+  p.gs_shift = 0;
+  while ((32 << p.gs_shift) < gs) ++p.gs_shift;
+  p.G = G;
+  p.U = U;
+  p.Upad = Upad;
+  p.PH = PH;
+  p.SLOTS = nsl;
+  p.RPT = RPT;
+  p.RT = RT;
+  p.RA = RA;
+  p.stages = static_cast<int>(ns);
+  p.wpr = wpr;
+  p.row_bytes = row_bytes;
+  p.w_stage = static_cast<uint32_t>(w_stage);
+  p.s_stage = static_cast<uint32_t>(s_stage);
+  const long long bars = ns * stage_bytes;
+  p.red_off = static_cast<uint32_t>((bars + 2 * ns * 8 + 15) / 16 * 16);
+  p.grp_off = static_cast<uint32_t>((p.red_off + red_bytes + 15) / 16 * 16);
+  pl.smem = static_cast<size_t>(p.grp_off + grp_bytes);
+  pl.mr = mr;
+  pl.nsl = nsl;
+  pl.threads = Tc + 32;
+  long long grid = dev->sms;
+  if (work_rows > 0 && work_rows < grid) grid = work_rows;
+  pl.grid = static_cast<int>(grid < 1 ? 1 : grid);
+  return QMV_OK;
+}
+
+template <int BITS, int MR, int NSL>
+int launch_t(const Plan &pl, cudaStream_t stream) {
+  auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL>;
+  // Raise the dynamic shared-memory limit to what this launch needs
+  // (idempotent; cheap compared with a launch).
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      static_cast<int>(pl.smem));
+  if (e != cudaSuccess)
+    return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+template <int BITS>
+int launch_bits(const Plan &pl, cudaStream_t stream) {
+  if (pl.nsl == 2) return launch_t<BITS, 1, 2>(pl, stream);
+  if (pl.mr == 2) return launch_t<BITS, 2, 1>(pl, stream);
+  return launch_t<BITS, 1, 1>(pl, stream);
+}
+
+int launch(const Plan &pl, int bits, cudaStream_t stream) {
+  switch (bits) {
+    case 2: return launch_bits<2>(pl, stream);
+    case 3: return launch_bits<3>(pl, stream);
+    case 4: return launch_bits<4>(pl, stream);
+    case 5: return launch_bits<5>(pl, stream);
+    case 6: return launch_bits<6>(pl, stream);
+    case 8: return launch_bits<8>(pl, stream);
+    default: return fail(QMV_ERR_UNSUPPORTED, "bits=%d", bits);
+  }
+}
+
+void init_params(qmvk::StreamParams &p) { std::memset(&p, 0, sizeof p); }
+
+}  // namespace
+
+extern "C" {
+
+int qmv_abi_version(void) { return 1; }
+
+const char *qmv_last_error(void) { return g_last_error.c_str(); }
+
+int qmv(const void *x, const uint32_t *w, const void *scales,
+        const void *biases, void *y, int M, int N, int K, int bits,
+        int group_size, void *stream) {
+  if (!x || !w || !scales || !biases || !y)
+    return fail(QMV_ERR_NULL, "qmv: a buffer pointer is NULL");
+  int rc = check_common(N, K, bits, group_size);
+  if (rc) return rc;
+  if (M <= 0) return fail(QMV_ERR_SHAPE, "qmv: M=%d must be positive", M);
+  if (!aligned16(x) || !aligned16(w) || !aligned16(scales) ||
+      !aligned16(biases) || !aligned16(y))
+    return fail(QMV_ERR_ALIGN, "qmv: buffers must be 16-byte aligned");
+  DeviceInfo *dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan pl;
+  init_params(pl.p);
+  qmvk::StreamParams &p = pl.p;
+  p.mode = qmvk::MODE_QMV;
+  p.w[0] = reinterpret_cast<const uint8_t *>(w);
+  p.s[0] = static_cast<const uint16_t *>(scales);
+  p.b[0] = static_cast<const uint16_t *>(biases);
+  p.y[0] = static_cast<uint16_t *>(y);
+  p.x = static_cast<const uint16_t *>(x);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nseg = 1;
+  p.total_rows = N;
+  if ((rc = make_plan(pl, bits, group_size, M, N, dev))) return rc;
+  return launch(pl, bits, static_cast<cudaStream_t>(stream));
+}
+
+int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
+                const void *b_gate, const uint32_t *w_up, const void *s_up,
+                const void *b_up, void *y_gate, void *y_up, int M, int N,
+                int K, int bits, int group_size, void *stream) {
+  if (!x || !w_gate || !s_gate || !b_gate || !w_up || !s_up || !b_up ||
+      !y_gate || !y_up)
+    return fail(QMV_ERR_NULL, "qmv_gate_up: a buffer pointer is NULL");
+  int rc = check_common(N, K, bits, group_size);
+  if (rc) return rc;
+  if (M <= 0) return fail(QMV_ERR_SHAPE, "qmv_gate_up: M=%d must be positive", M);
+  const void *ptrs[] = {x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up};
+  for (const void *q : ptrs)
+    if (!aligned16(q))
+      return fail(QMV_ERR_ALIGN, "qmv_gate_up: buffers must be 16-byte aligned");
+  DeviceInfo *dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan pl;
+  init_params(pl.p);
+  qmvk::StreamParams &p = pl.p;
+  p.mode = qmvk::MODE_GATE_UP;
+  p.w[0] = reinterpret_cast<const uint8_t *>(w_gate);
+  p.s[0] = static_cast<const uint16_t *>(s_gate);
+  p.b[0] = static_cast<const uint16_t *>(b_gate);
+  p.y[0] = static_cast<uint16_t *>(y_gate);
+  p.w[1] = reinterpret_cast<const uint8_t *>(w_up);
+  p.s[1] = static_cast<const uint16_t *>(s_up);
+  p.b[1] = static_cast<const uint16_t *>(b_up);
+  p.y[1] = static_cast<uint16_t *>(y_up);
+  p.x = static_cast<const uint16_t *>(x);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nseg = 2;
+  p.total_rows = N;
+  if ((rc = make_plan(pl, bits, group_size, M, 2LL * N, dev))) return rc;
+  return launch(pl, bits, static_cast<cudaStream_t>(stream));
+}
+
+int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
+                        const uint32_t *w, const void *scales,
+                        const void *biases, void *y, int M, int N, int K,
+                        int bits, int group_size, void *stream) {
+  if (!gate || !up || !w || !scales || !biases || !y)
+    return fail(QMV_ERR_NULL, "qmv_silu_gate_resid: a buffer pointer is NULL");
+  int rc = check_common(N, K, bits, group_size);
+  if (rc) return rc;
+  if (M <= 0)
+    return fail(QMV_ERR_SHAPE, "qmv_silu_gate_resid: M=%d must be positive", M);
+  const void *ptrs[] = {gate, up, w, scales, biases, y};
+  for (const void *q : ptrs)
+    if (!aligned16(q))
+      return fail(QMV_ERR_ALIGN,
+                  "qmv_silu_gate_resid: buffers must be 16-byte aligned");
+  if (x_resid && (reinterpret_cast<uintptr_t>(x_resid) & 1u))
+    return fail(QMV_ERR_ALIGN, "qmv_silu_gate_resid: x_resid must be 2-byte aligned");
+  DeviceInfo *dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan pl;
+  init_params(pl.p);
+  qmvk::StreamParams &p = pl.p;
+  p.mode = qmvk::MODE_SILU;
+  p.w[0] = reinterpret_cast<const uint8_t *>(w);
+  p.s[0] = static_cast<const uint16_t *>(scales);
+  p.b[0] = static_cast<const uint16_t *>(biases);
+  p.y[0] = static_cast<uint16_t *>(y);
+  p.x = static_cast<const uint16_t *>(gate);
+  p.up = static_cast<const uint16_t *>(up);
+  p.resid = static_cast<const uint16_t *>(x_resid);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nseg = 1;
+  p.total_rows = N;
+  if ((rc = make_plan(pl, bits, group_size, M, N, dev))) return rc;
+  return launch(pl, bits, static_cast<cudaStream_t>(stream));
+}
+
+int gather_qmv(const void *x, const uint32_t *w, const void *scales,
+               const void *biases, const uint32_t *lhs_indices,
+               const uint32_t *rhs_indices, void *y, int num_pairs,
+               int num_x_rows, int num_experts, int N, int K, int bits,
+               int group_size, int sorted_indices, int *d_status,
+               void *stream) {
+  (void)sorted_indices;  // grouping by expert happens on the device either way
+  if (!x || !w || !scales || !biases || !rhs_indices || !y)
+    return fail(QMV_ERR_NULL, "gather_qmv: a buffer pointer is NULL");
+  int rc = check_common(N, K, bits, group_size);
+  if (rc) return rc;
+  if (num_pairs < 0 || num_x_rows <= 0 || num_experts <= 0)
+    return fail(QMV_ERR_SHAPE,
+                "gather_qmv: num_pairs=%d num_x_rows=%d num_experts=%d",
+                num_pairs, num_x_rows, num_experts);
+  if (!lhs_indices && num_x_rows < num_pairs)
+    return fail(QMV_ERR_SHAPE,
+                "gather_qmv: without lhs_indices num_x_rows must be >= num_pairs");
+  if (3LL * num_experts + num_pairs > 24576)
+    return fail(QMV_ERR_UNSUPPORTED,
+                "gather_qmv: num_pairs + 3*num_experts above 24576");
+  if (num_pairs == 0) return ok();
+  const void *ptrs[] = {x, w, scales, biases, y};
+  for (const void *q : ptrs)
+    if (!aligned16(q))
+      return fail(QMV_ERR_ALIGN, "gather_qmv: buffers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(rhs_indices) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lhs_indices) & 3u) ||
+      (reinterpret_cast<uintptr_t>(d_status) & 3u))
+    return fail(QMV_ERR_ALIGN, "gather_qmv: index arrays must be 4-byte aligned");
+  DeviceInfo *dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan pl;
+  init_params(pl.p);
+  qmvk::StreamParams &p = pl.p;
+  p.mode = qmvk::MODE_GATHER;
+  p.w[0] = reinterpret_cast<const uint8_t *>(w);
+  p.s[0] = static_cast<const uint16_t *>(scales);
+  p.b[0] = static_cast<const uint16_t *>(biases);
+  p.y[0] = static_cast<uint16_t *>(y);
+  p.x = static_cast<const uint16_t *>(x);
+  p.lhs = lhs_indices;
+  p.rhs = rhs_indices;
+  p.status = d_status;
+  p.M = 1;
+  p.N = N;
+  p.K = K;
+  p.nseg = 1;
+  p.total_rows = static_cast<long long>(num_experts) * N;
+  p.num_pairs = num_pairs;
+  p.num_x_rows = num_x_rows;
+  p.num_experts = num_experts;
+  const int mr = num_pairs >= num_experts ? 2 : 1;
+  if ((rc = make_plan(pl, bits, group_size, mr, 0, dev))) return rc;
+  return launch(pl, bits, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+/*
+ * qmv.h -- C ABI of libqmv, the B200 (sm_100a) affine group-quantized
+ * matrix-vector product and its fused decode variants.
+ *
+ * ---------------------------------------------------------------------------
+ * Data format (shared by every entry point)
+ * ---------------------------------------------------------------------------
+ * A quantized weight W has N rows and K columns.  Each row is one packed,
+ * unpadded bitstream of K codes of `bits` bits, least-significant bit first,
+ * stored as K*bits/32 uint32 words (row byte stride K*bits/8).  Code k of a
+ * row occupies bits [k*bits, (k+1)*bits) of the row's little-endian byte
+ * string.  This is the layout of the pages' pack-factor helpers and
+ * affine_dequantize kernel ("mlx/include/mlx/backend/metal/kernels/
+ * quantized.h", MLX 0.30.1): 2/4/8-bit pack 16/8/4 codes per word, 3-bit 8
+ * codes per 3 bytes, 5-bit 8 codes per 5 bytes, 6-bit 4 codes per 3 bytes.
+ *
+ * scales and biases are bf16 [N, K/group_size]; group g of row n covers
+ * columns [g*group_size, (g+1)*group_size) and dequantizes as
+ *     w_hat[n][k] = scale[n][g] * q[n][k] + bias[n][g]
+ * (same page, affine_dequantize and qdot).  Scales may be negative.
+ *
+ * All activations and outputs are bf16 (passed as void*, uint16 bit
+ * patterns), row-major and contiguous.  Arithmetic is fp32 with one final
+ * round-to-nearest-even to bf16.
+ *
+ * Supported: bits in {2,3,4,5,6,8}; group_size in {32,64,128}; K a positive
+ * multiple of group_size; N >= 1; M >= 1.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions
+ * ---------------------------------------------------------------------------
+ * Pointers: every buffer pointer is a DEVICE pointer owned by the caller and
+ * must be 16-byte aligned.  The library never frees or retains them and does
+ * not allocate device memory.
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * Every call only enqueues work on that stream and returns; results are
+ * ready when the stream is synchronized.  Each successful call enqueues
+ * exactly one kernel.
+ * Errors: every argument is checked on the host before anything is
+ * enqueued; on a bad argument nothing touches the device and the call
+ * returns a nonzero qmv_status.  qmv_last_error() then describes the failure
+ * (thread-local; valid until the next call on the same thread).  There is no
+ * silent fallback: a combination without a kernel returns
+ * QMV_ERR_UNSUPPORTED (the pages' QuantWeights trait makes its fused
+ * operations return an error rather than take a slow path).
+ */
+#ifndef LIBQMV_QMV_H
+#define LIBQMV_QMV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QMV_OK = 0,
+    QMV_ERR_NULL = 1,        /* a required pointer is NULL                   */
+    QMV_ERR_SHAPE = 2,       /* M, N, K, counts or group layout inconsistent */
+    QMV_ERR_UNSUPPORTED = 3, /* bits / group_size outside the supported set  */
+    QMV_ERR_ALIGN = 4,       /* a buffer pointer is not 16-byte aligned      */
+    QMV_ERR_CUDA = 5         /* a CUDA runtime call or launch failed         */
+} qmv_status;
+
+/*
+ * qmv -- y = x @ dequant(W).T
+ *
+ * Defined by the pages' quantized_matmul with transpose = true
+ * ("mlx/include/mlx/backend/metal/kernels/quantized.h": qmv / qmv_fast) and
+ * by the QuantWeights trait's gemv ("decode matvec y = self @ x").
+ *   x       bf16 [M, K]
+ *   w       uint32 [N, K*bits/32]  (packed rows, layout above)
+ *   scales  bf16 [N, K/group_size]
+ *   biases  bf16 [N, K/group_size]
+ *   y       bf16 [M, N]  (written; must not overlap the inputs)
+ *   y[m][n] = sum_k x[m][k] * w_hat[n][k]
+ */
+int qmv(const void *x, const uint32_t *w, const void *scales,
+        const void *biases, void *y, int M, int N, int K, int bits,
+        int group_size, void *stream);
+
+/*
+ * qmv_gate_up -- dual-output GEMV over one input, in ONE kernel launch:
+ *   y_gate = x @ dequant(W_gate).T,   y_up = x @ dequant(W_up).T
+ *
+ * Defined by the QuantWeights trait's gemv_gate_up_with (pages
+ * "QuantWeights" and "quant_weights.rs"): two matrices of the same shape
+ * (the trait asserts equal in/out features), each with its own scales and
+ * biases, one shared x.
+ *   x                         bf16 [M, K]
+ *   w_gate, w_up              uint32 [N, K*bits/32]
+ *   s_gate, b_gate, s_up, b_up  bf16 [N, K/group_size]
+ *   y_gate, y_up              bf16 [M, N]
+ */
+int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
+                const void *b_gate, const uint32_t *w_up, const void *s_up,
+                const void *b_up, void *y_gate, void *y_up, int M, int N,
+                int K, int bits, int group_size, void *stream);
+
+/*
+ * qmv_silu_gate_resid -- fused FFN tail with the residual add folded in:
+ *   y[m][n] = x_resid[m][n] + sum_k w_hat[n][k] * silu(gate[m][k]) * up[m][k]
+ *
+ * Defined by the QuantWeights trait's gemv_silu_gate_resid; with
+ * x_resid == NULL it is gemv_silu_gate (y = W @ (silu(gate) * up)).
+ * silu(g) = g / (1 + exp(-g)).  silu(gate)*up is formed in fp32 inside the
+ * kernel and is never rounded to bf16.
+ *   gate, up   bf16 [M, K]
+ *   x_resid    bf16 [M, N] or NULL
+ *   w          uint32 [N, K*bits/32]; scales, biases bf16 [N, K/group_size]
+ *   y          bf16 [M, N]
+ */
+int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
+                        const uint32_t *w, const void *scales,
+                        const void *biases, void *y, int M, int N, int K,
+                        int bits, int group_size, void *stream);
+
+/*
+ * gather_qmv -- index-gathered per-expert GEMV:
+ *   y[p] = x[lhs_indices[p]] @ dequant(W[rhs_indices[p]]).T,  p < num_pairs
+ *
+ * Defined by the pages' gather_qmm ("mlx.core.gather_qmm": lhs_indices and
+ * rhs_indices are flat indices into the batch dimensions of x and w;
+ * sorted_indices "may allow a faster implementation") and by the gather
+ * form of adjust_matrix_offsets in quantized.h.
+ *   x            bf16 [num_x_rows, K]
+ *   w            uint32 [num_experts, N, K*bits/32]
+ *   scales/biases bf16 [num_experts, N, K/group_size]
+ *   lhs_indices  uint32 [num_pairs] device array, or NULL (pair p reads x row p;
+ *                then num_x_rows must be >= num_pairs)
+ *   rhs_indices  uint32 [num_pairs] device array (expert of pair p)
+ *   y            bf16 [num_pairs, N]
+ *   sorted_indices  nonzero when rhs_indices is non-decreasing.  A hint
+ *                only: the value of every output row is the same either way
+ *                (bit-identical), whatever the order of the pairs.
+ *   d_status     device int or NULL.  If any index is out of range the
+ *                kernel ORs 1 into *d_status and leaves that pair's output
+ *                row unwritten; valid pairs are still computed.  The caller
+ *                zeroes *d_status before the call.
+ * The kernel reads every expert that some pair uses once per call, whether or
+ * not the indices are sorted.  num_pairs may be 0 (nothing is enqueued).
+ */
+int gather_qmv(const void *x, const uint32_t *w, const void *scales,
+               const void *biases, const uint32_t *lhs_indices,
+               const uint32_t *rhs_indices, void *y, int num_pairs,
+               int num_x_rows, int num_experts, int N, int K, int bits,
+               int group_size, int sorted_indices, int *d_status,
+               void *stream);
+
+/* Message for the last non-OK return on this thread ("" if none). */
+const char *qmv_last_error(void);
+
+/* ABI version of this header (incremented on incompatible change). */
+int qmv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBQMV_QMV_H */
