@@ -110,98 +110,122 @@ struct Plan {
   int grid = 0;
 };
 
-int make_plan(Plan &pl, int bits, int gs, int mr_want, long long work_rows,
-              DeviceInfo *dev) {
+// Rows per consumer thread per tile; the same rule as the kernel's
+// rows_per_thread<BITS, MR, NSL>().
+int rows_per_thread_host(int bits, int mr, int nsl) {
+  const int base = bits == 2 ? 16 : (bits == 3 || bits == 4) ? 8 : 4;
+  return (mr * nsl == 1) ? base : (base / 2 < 2 ? 2 : base / 2);
+}
+
+// Thread layout: Upad (>= 32, a multiple of 32) consumer threads cover the
+// 32-code units of one row, PH such groups work on PH rows at once; each
+// consumer thread handles RPT rows of its unit per tile.  One epilogue warp
+// completes the CTA.
+int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   qmvk::StreamParams &p = pl.p;
   const int K = p.K;
   const int U = K / 32;
-  int Upad, nsl = 1, PH = 1;
-  if (U >= 32) {
-    Upad = (U + 31) / 32 * 32;
-  } else {
-    Upad = 1;
-    while (Upad < U) Upad <<= 1;
-  }
+  int Upad = U < 32 ? 32 : (U + 31) / 32 * 32;
+  int nsl = 1;
   if (Upad > 448) {
     Upad = (U + 63) / 64 * 64;
     nsl = 2;
-  } else {
-    PH = Upad <= 256 ? (256 + Upad - 1) / Upad : 1;
   }
-  const int Tc = Upad * PH / nsl;
-  if (Tc > 448 || Tc % 32 != 0)
-    return fail(QMV_ERR_UNSUPPORTED, "K=%d has no thread layout", K);
-  const int L = Upad < 32 ? Upad : 32;
-  const int mr = (nsl == 1 && mr_want >= 2 && L >= 2) ? 2 : 1;
+  const int mr = (nsl == 1 && mr_want >= 2) ? 2 : 1;
   const long long row_bytes = static_cast<long long>(K) * bits / 8;
   const int G = K / gs;
-  // rows per thread per tile: largest power of two with RPT*MR <= L that
-  // keeps one stage's weight bytes within 32 KB
-  int RPT = 8;
-  while (RPT > 1 && (RPT * mr > L || static_cast<long long>(RPT) * PH * row_bytes > 32768))
-    RPT >>= 1;
-  const int RT = RPT * PH;
-  const int ra_w = 16 / gcd_i(static_cast<int>(row_bytes % 16 == 0 ? 16 : row_bytes % 16), 16);
-  const int ra_s = 16 / gcd_i((2 * G) % 16 == 0 ? 16 : (2 * G) % 16, 16);
-  const int RA = ra_w * ra_s / gcd_i(ra_w, ra_s);
-  const long long stage_rows = RT + RA - 1;
-  const long long w_stage = (stage_rows * row_bytes + 15 + 15) / 16 * 16;
-  const long long s_stage = (stage_rows * 2LL * G + 15 + 15) / 16 * 16;
-  const long long stage_bytes = w_stage + 2 * s_stage;
-  const int wpr = Upad >= 32 ? Upad / 32 / nsl : 1;
-  const long long red_bytes = 2LL * RT * mr * wpr * 4;
+  const int RPT = rows_per_thread_host(bits, mr, nsl);
   long long grp_bytes = 0;
   if (p.mode == qmvk::MODE_GATHER)
-    grp_bytes = (3LL * p.num_experts + 1 + p.num_pairs) * 4;
-  const long long budget = dev->smem_optin;
-  const long long fixed = 2LL * 8 * 8 + red_bytes + grp_bytes + 256;
-  long long ns = (budget - fixed) / stage_bytes;
-  if (ns > 8) ns = 8;
-  if (ns < 2)
-    return fail(QMV_ERR_UNSUPPORTED,
-                "shape needs more shared memory than the device offers "
-                "(stage %lld B, fixed %lld B)",
-                stage_bytes, fixed);
+    grp_bytes = (2LL * p.num_experts + 3LL * p.num_pairs + 1) * 4;
+  // consumer threads: up to 448 (plus one epilogue warp: 480 per CTA, so
+  // that every thread can hold 128 registers), as many row phases as keep a
+  // copy ring at least three tiles deep (two at the least)
+  const int tc_max = 448;
+  int PH = nsl == 1 && Upad <= tc_max ? tc_max / Upad : 1;
+  auto ring_depth = [&](int ph) {
+    const long long tc = static_cast<long long>(Upad) * ph / nsl;
+    const long long rt = static_cast<long long>(RPT) * ph;
+    const long long red = 4 * ((rt * mr * (Upad / 32 / nsl) * 4 + 15) / 16 * 16);
+    const long long fixed = red + 64 + grp_bytes + 256;
+    const long long stage = RPT * nsl * tc * (4LL * bits + 8);
+    return (dev->smem_optin - fixed) / stage;
+  };
+  while (PH > 1 && ring_depth(PH) < 3) --PH;
+  const int Tc = Upad * PH / nsl;
+  if (Tc > tc_max || Tc % 32 != 0)
+    return fail(QMV_ERR_UNSUPPORTED, "K=%d has no thread layout", K);
+  const int RT = RPT * PH;
+  const int wpr = Upad / 32 / nsl;
+  const int nred = 4;
+  const long long red_slot = (static_cast<long long>(RT) * mr * wpr * 4 + 15) / 16 * 16;
+  const long long bar_off = nred * red_slot;
+  const long long grp_off = (bar_off + 2 * nred * 8 + 15) / 16 * 16;
+  const long long cp_off = (grp_off + grp_bytes + 127) / 128 * 128;
+  // copy ring: depth stages of RPT rows x units x (unit bytes + scale/bias)
+  const long long stage = static_cast<long long>(RPT) * nsl * Tc * (4LL * bits + 8);
+  long long depth = (dev->smem_optin - cp_off) / stage;
+  if (depth > 4) depth = 4;
+  if (depth < 2)
+    return fail(QMV_ERR_UNSUPPORTED, "shape needs more shared memory than the device offers");
+  const long long smem = cp_off + depth * stage;
   p.gs_shift = 0;
   while ((32 << p.gs_shift) < gs) ++p.gs_shift;
   p.G = G;
   p.U = U;
   p.Upad = Upad;
   p.PH = PH;
-  p.SLOTS = nsl;
-  p.RPT = RPT;
   p.RT = RT;
-  p.RA = RA;
-  p.stages = static_cast<int>(ns);
+  p.nred = nred;
   p.wpr = wpr;
-  p.row_bytes = row_bytes;
-  p.w_stage = static_cast<uint32_t>(w_stage);
-  p.s_stage = static_cast<uint32_t>(s_stage);
-  const long long bars = ns * stage_bytes;
-  p.red_off = static_cast<uint32_t>((bars + 2 * ns * 8 + 15) / 16 * 16);
-  p.grp_off = static_cast<uint32_t>((p.red_off + red_bytes + 15) / 16 * 16);
-  pl.smem = static_cast<size_t>(p.grp_off + grp_bytes);
+  p.row_bytes = static_cast<uint32_t>(row_bytes);
+  p.nch = p.mode == qmvk::MODE_GATHER ? 1 : (p.M + mr - 1) / mr;
+  p.red_off = 0;
+  p.red_slot = static_cast<uint32_t>(red_slot);
+  p.bar_off = static_cast<uint32_t>(bar_off);
+  p.grp_off = static_cast<uint32_t>(grp_off);
+  p.cp_off = static_cast<uint32_t>(cp_off);
+  p.depth = static_cast<int>(depth);
+  p.sb_pairs = (G % 2 == 0) ? 1 : 0;
+  pl.smem = static_cast<size_t>(smem);
   pl.mr = mr;
   pl.nsl = nsl;
   pl.threads = Tc + 32;
+  // one CTA per SM; fewer when there is less work than SMs
+  long long work = p.mode == qmvk::MODE_GATHER
+                       ? static_cast<long long>(dev->sms)
+                       : static_cast<long long>(p.nmat) * p.nch * p.N;
+  if (work > 0x7fffffffLL)
+    return fail(QMV_ERR_UNSUPPORTED, "too many output rows in one call");
   long long grid = dev->sms;
-  if (work_rows > 0 && work_rows < grid) grid = work_rows;
+  if (work < grid) grid = work;
   pl.grid = static_cast<int>(grid < 1 ? 1 : grid);
   return QMV_OK;
 }
 
 template <int BITS, int MR, int NSL>
+int &granted_smem(int dev) {
+  static int granted[kMaxDevices] = {};
+  return granted[dev];
+}
+
+template <int BITS, int MR, int NSL>
 int launch_t(const Plan &pl, cudaStream_t stream) {
   auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL>;
-  // Raise the dynamic shared-memory limit to what this launch needs
-  // (idempotent; cheap compared with a launch).
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      static_cast<int>(pl.smem));
-  if (e != cudaSuccess)
-    return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &granted = granted_smem<BITS, MR, NSL>(dev);
+  if (static_cast<int>(pl.smem) > granted) {
+    cudaError_t e = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        static_cast<int>(pl.smem));
+    if (e != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s",
+                  cudaGetErrorString(e));
+    granted = static_cast<int>(pl.smem);
+  }
   kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.p);
-  e = cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
   return ok();
@@ -261,9 +285,8 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.nseg = 1;
-  p.total_rows = N;
-  if ((rc = make_plan(pl, bits, group_size, M, N, dev))) return rc;
+  p.nmat = 1;
+  if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
 
@@ -277,6 +300,8 @@ int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
   int rc = check_common(N, K, bits, group_size);
   if (rc) return rc;
   if (M <= 0) return fail(QMV_ERR_SHAPE, "qmv_gate_up: M=%d must be positive", M);
+  if (N > (1 << 30))
+    return fail(QMV_ERR_UNSUPPORTED, "qmv_gate_up: N=%d above 2^30", N);
   const void *ptrs[] = {x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up};
   for (const void *q : ptrs)
     if (!aligned16(q))
@@ -299,9 +324,8 @@ int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.nseg = 2;
-  p.total_rows = N;
-  if ((rc = make_plan(pl, bits, group_size, M, 2LL * N, dev))) return rc;
+  p.nmat = 2;
+  if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
 
@@ -338,9 +362,8 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.nseg = 1;
-  p.total_rows = N;
-  if ((rc = make_plan(pl, bits, group_size, M, N, dev))) return rc;
+  p.nmat = 1;
+  if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
 
@@ -362,6 +385,8 @@ int gather_qmv(const void *x, const uint32_t *w, const void *scales,
   if (!lhs_indices && num_x_rows < num_pairs)
     return fail(QMV_ERR_SHAPE,
                 "gather_qmv: without lhs_indices num_x_rows must be >= num_pairs");
+  if (static_cast<long long>(num_experts) * N > 0x7fffffffLL)
+    return fail(QMV_ERR_UNSUPPORTED, "gather_qmv: num_experts * N above 2^31");
   if (3LL * num_experts + num_pairs > 24576)
     return fail(QMV_ERR_UNSUPPORTED,
                 "gather_qmv: num_pairs + 3*num_experts above 24576");
@@ -391,13 +416,12 @@ int gather_qmv(const void *x, const uint32_t *w, const void *scales,
   p.M = 1;
   p.N = N;
   p.K = K;
-  p.nseg = 1;
-  p.total_rows = static_cast<long long>(num_experts) * N;
+  p.nmat = 1;
   p.num_pairs = num_pairs;
   p.num_x_rows = num_x_rows;
   p.num_experts = num_experts;
   const int mr = num_pairs >= num_experts ? 2 : 1;
-  if ((rc = make_plan(pl, bits, group_size, mr, 0, dev))) return rc;
+  if ((rc = make_plan(pl, bits, group_size, mr, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
 

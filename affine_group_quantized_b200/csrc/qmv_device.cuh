@@ -172,31 +172,49 @@ __device__ __forceinline__ float code_as_float(const uint32_t (&wd)[BITS]) {
   return __uint_as_float(v & mask);
 }
 
+// Two rows of one unit at a time: the codes of both rows are decoded and fed
+// to fp32 FMAs against the same pre-scaled activations.  Each row keeps four
+// accumulators, so the eight FMA chains of a row pair are independent and the
+// decode instructions interleave with them.
 template <int BITS, int MR, int J>
-__device__ __forceinline__ void fma_code_pair(const uint32_t (&wd)[BITS],
-                                              const float2 (&xp)[MR][16],
-                                              float2 (&acc)[MR]) {
-  const float2 f = make_float2(code_as_float<BITS, 2 * J>(wd),
-                               code_as_float<BITS, 2 * J + 1>(wd));
+__device__ __forceinline__ void fma_pair_2rows(const uint32_t (&w0)[BITS],
+                                               const uint32_t (&w1)[BITS],
+                                               const float2 (&xp)[MR][16],
+                                               float2 (&a0)[MR][2],
+                                               float2 (&a1)[MR][2]) {
+  // scalar FMAs: packed fp32x2 FMAs would need the two decoded codes moved
+  // into a register pair first, which costs more than it saves
+  const float f0x = code_as_float<BITS, 2 * J>(w0);
+  const float f0y = code_as_float<BITS, 2 * J + 1>(w0);
+  const float f1x = code_as_float<BITS, 2 * J>(w1);
+  const float f1y = code_as_float<BITS, 2 * J + 1>(w1);
 #pragma unroll
-  for (int m = 0; m < MR; ++m) acc[m] = __ffma2_rn(f, xp[m][J], acc[m]);
+  for (int m = 0; m < MR; ++m) {
+    a0[m][J & 1].x = fmaf(f0x, xp[m][J].x, a0[m][J & 1].x);
+    a0[m][J & 1].y = fmaf(f0y, xp[m][J].y, a0[m][J & 1].y);
+    a1[m][J & 1].x = fmaf(f1x, xp[m][J].x, a1[m][J & 1].x);
+    a1[m][J & 1].y = fmaf(f1y, xp[m][J].y, a1[m][J & 1].y);
+  }
 }
 
 template <int BITS, int MR, int... J>
-__device__ __forceinline__ void unit_fma_impl(const uint32_t (&wd)[BITS],
-                                              const float2 (&xp)[MR][16],
-                                              float2 (&acc)[MR],
-                                              std::integer_sequence<int, J...>) {
-  (fma_code_pair<BITS, MR, J>(wd, xp, acc), ...);
+__device__ __forceinline__ void unit_fma_2rows_impl(
+    const uint32_t (&w0)[BITS], const uint32_t (&w1)[BITS],
+    const float2 (&xp)[MR][16], float2 (&a0)[MR][2], float2 (&a1)[MR][2],
+    std::integer_sequence<int, J...>) {
+  (fma_pair_2rows<BITS, MR, J>(w0, w1, xp, a0, a1), ...);
 }
 
-// acc[m] += sum_i x''[m][i] * f_i over the 32 codes of one unit (two fp32
-// lanes per accumulator; caller adds .x + .y).
+// a{0,1}[m][*] += x''[m][i] * f_i over the 32 codes of one unit of rows 0/1.
+// The caller sums the four fp32 lanes of each row.
 template <int BITS, int MR>
-__device__ __forceinline__ void unit_fma(const uint32_t (&wd)[BITS],
-                                         const float2 (&xp)[MR][16],
-                                         float2 (&acc)[MR]) {
-  unit_fma_impl<BITS, MR>(wd, xp, acc, std::make_integer_sequence<int, 16>{});
+__device__ __forceinline__ void unit_fma_2rows(const uint32_t (&w0)[BITS],
+                                               const uint32_t (&w1)[BITS],
+                                               const float2 (&xp)[MR][16],
+                                               float2 (&a0)[MR][2],
+                                               float2 (&a1)[MR][2]) {
+  unit_fma_2rows_impl<BITS, MR>(w0, w1, xp, a0, a1,
+                                std::make_integer_sequence<int, 16>{});
 }
 
 // Load one unit (BITS words) from shared memory, using the widest aligned
@@ -251,6 +269,149 @@ __device__ __forceinline__ void prescale_unit(const float (&v)[32],
     const float a = v[2 * j] * pow2i(149 - code_pos(BITS, 2 * j) - c);
     const float b = v[2 * j + 1] * pow2i(149 - code_pos(BITS, 2 * j + 1) - c);
     xp[j] = make_float2(a, b);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Integer path for 2-, 4- and 8-bit codes.
+//
+// The 32 codes of a unit are spread into eight 32-bit registers holding four
+// codes each, one per byte (8-bit: the words themselves; 4-bit: the even and
+// the odd nibbles of each word, masked; 2-bit: the four 2-bit lanes of each
+// byte, shifted and masked).  The activations of the unit are turned into
+// 22-bit fixed point relative to the unit's largest magnitude,
+// X_i = rint(x_i * 2^s) with |X_i| <= 2^22, and X_i is split into three
+// signed 8-bit digits: X = L2 * 2^16 + L1 * 2^8 + L0.  Every digit register
+// holds the digits of the four activations that meet the four codes of one
+// code register, so dp4a (four 8-bit products added to a 32-bit integer)
+// computes sum_i q_i * L_i exactly.  X_i equals x_i * 2^s exactly whenever
+// |x_i| is within 2^14 of the unit's largest |x| (a bf16 carries 8
+// significant bits); smaller elements are rounded to the unit's grid, an
+// error below 2^-23 of the unit's largest |x|.
+// Each digit sum starts from 0x4B400000, the bit pattern of 1.5 * 2^23: as
+// long as |sum| < 2^22 the 32-bit result read as a float is 1.5 * 2^23 + sum
+// exactly, so no integer-to-float conversion is needed.
+// ---------------------------------------------------------------------------
+
+template <int BITS>
+constexpr bool kIntPath = BITS == 2 || BITS == 4 || BITS == 8;
+
+constexpr int kDigitBias = 0x4B400000;        // bits of 12582912.0f
+constexpr float kDigitBiasF = 12582912.0f;
+
+// (register, byte lane) of code i of a unit in the spread layout
+__host__ __device__ constexpr int spread_reg(int bits, int i) {
+  return bits == 8 ? i / 4
+       : bits == 4 ? 2 * (i / 8) + (i % 8) % 2
+                   : 4 * (i / 16) + (i % 16) % 4;
+}
+__host__ __device__ constexpr int spread_lane(int bits, int i) {
+  return bits == 8 ? i % 4 : bits == 4 ? (i % 8) / 2 : (i % 16) / 4;
+}
+
+// Spread register r (0..7) of a unit: four codes, one per byte.
+template <int BITS, int R>
+__device__ __forceinline__ uint32_t spread_codes(const uint32_t (&wd)[BITS]) {
+  if constexpr (BITS == 8) {
+    return wd[R];
+  } else if constexpr (BITS == 4) {
+    const uint32_t w = wd[R / 2];
+    return (R % 2 == 0 ? w : (w >> 4)) & 0x0F0F0F0Fu;
+  } else {
+    const uint32_t w = wd[R / 4];
+    return (w >> (2 * (R % 4))) & 0x03030303u;
+  }
+}
+
+__device__ __forceinline__ int dp4a_su(int a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Digits of the unit's activations in the spread layout, the scale back to
+// activation units (2^-s) and the plain activation sum times 2^s.
+template <int BITS>
+__device__ __forceinline__ void digits_unit(const float (&v)[32],
+                                            int (&dig)[3][8], float &inv,
+                                            float &vs) {
+  float mx = 0.f, sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    mx = fmaxf(mx, fabsf(v[i]));
+    sum += v[i];
+  }
+  const int eb = static_cast<int>((__float_as_uint(mx) >> 23) & 0xff);
+  int s = 148 - eb;  // max|v| < 2^(eb-126), so |v| * 2^s < 2^22
+  s = s < -126 ? -126 : (s > 126 ? 126 : s);
+  const float sc = pow2i(s);
+  inv = pow2i(-s);
+  vs = sum * sc;
+#pragma unroll
+  for (int l = 0; l < 3; ++l)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) dig[l][r] = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int X = __float2int_rn(v[i] * sc);
+    const int L0 = static_cast<int>(static_cast<int8_t>(X & 0xff));
+    const int X1 = (X - L0) >> 8;
+    const int L1 = static_cast<int>(static_cast<int8_t>(X1 & 0xff));
+    const int L2 = (X1 - L1) >> 8;
+    const int r = spread_reg(BITS, i), sh = 8 * spread_lane(BITS, i);
+    dig[0][r] |= (L0 & 0xff) << sh;
+    dig[1][r] |= (L1 & 0xff) << sh;
+    dig[2][r] |= (L2 & 0xff) << sh;
+  }
+}
+
+template <int BITS, int MR, int R>
+__device__ __forceinline__ void dp_reg_2rows(const uint32_t (&w0)[BITS],
+                                             const uint32_t (&w1)[BITS],
+                                             const int (&dig)[MR][3][8],
+                                             int (&a0)[MR][3], int (&a1)[MR][3]) {
+  const uint32_t b0 = spread_codes<BITS, R>(w0);
+  const uint32_t b1 = spread_codes<BITS, R>(w1);
+#pragma unroll
+  for (int m = 0; m < MR; ++m)
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      a0[m][l] = dp4a_su(dig[m][l][R], b0, a0[m][l]);
+      a1[m][l] = dp4a_su(dig[m][l][R], b1, a1[m][l]);
+    }
+}
+
+template <int BITS, int MR, int... R>
+__device__ __forceinline__ void unit_dp_2rows_impl(
+    const uint32_t (&w0)[BITS], const uint32_t (&w1)[BITS],
+    const int (&dig)[MR][3][8], int (&a0)[MR][3], int (&a1)[MR][3],
+    std::integer_sequence<int, R...>) {
+  (dp_reg_2rows<BITS, MR, R>(w0, w1, dig, a0, a1), ...);
+}
+
+// sum_i q_i * X_i of one unit for two rows, as floats (exact up to the last
+// two additions).
+template <int BITS, int MR>
+__device__ __forceinline__ void unit_dp_2rows(const uint32_t (&w0)[BITS],
+                                              const uint32_t (&w1)[BITS],
+                                              const int (&dig)[MR][3][8],
+                                              float (&r0)[MR], float (&r1)[MR]) {
+  int a0[MR][3], a1[MR][3];
+#pragma unroll
+  for (int m = 0; m < MR; ++m)
+#pragma unroll
+    for (int l = 0; l < 3; ++l) a0[m][l] = a1[m][l] = kDigitBias;
+  unit_dp_2rows_impl<BITS, MR>(w0, w1, dig, a0, a1,
+                               std::make_integer_sequence<int, 8>{});
+#pragma unroll
+  for (int m = 0; m < MR; ++m) {
+    r0[m] = fmaf(__int_as_float(a0[m][2]) - kDigitBiasF, 65536.f,
+                 fmaf(__int_as_float(a0[m][1]) - kDigitBiasF, 256.f,
+                      __int_as_float(a0[m][0]) - kDigitBiasF));
+    r1[m] = fmaf(__int_as_float(a1[m][2]) - kDigitBiasF, 65536.f,
+                 fmaf(__int_as_float(a1[m][1]) - kDigitBiasF, 256.f,
+                      __int_as_float(a1[m][0]) - kDigitBiasF));
   }
 }
 
