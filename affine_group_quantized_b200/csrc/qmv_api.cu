@@ -119,8 +119,9 @@ int rows_per_thread_host(int bits, int mr, int nsl) {
 
 // Thread layout: Upad (>= 32, a multiple of 32) consumer threads cover the
 // 32-code units of one row, PH such groups work on PH rows at once; each
-// consumer thread handles RPT rows of its unit per tile.  One epilogue warp
-// completes the CTA.
+// consumer thread handles up to RPT rows of its unit per tile.  A producer
+// warp and an epilogue warp complete the CTA.  Stages hold RT rows (plus the
+// rows copied only for alignment) of weights, scales and biases.
 int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   qmvk::StreamParams &p = pl.p;
   const int K = p.K;
@@ -138,37 +139,40 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   long long grp_bytes = 0;
   if (p.mode == qmvk::MODE_GATHER)
     grp_bytes = (2LL * p.num_experts + 3LL * p.num_pairs + 1) * 4;
-  // consumer threads: up to 448 (plus one epilogue warp: 480 per CTA, so
-  // that every thread can hold 128 registers), as many row phases as keep a
-  // copy ring at least three tiles deep (two at the least)
+  const int ra_w = 16 / gcd_i(static_cast<int>(row_bytes % 16 == 0 ? 16 : row_bytes % 16), 16);
+  const int ra_s = 16 / gcd_i((2 * G) % 16 == 0 ? 16 : (2 * G) % 16, 16);
+  const int RA = ra_w * ra_s / gcd_i(ra_w, ra_s);
+  const int wpr = Upad / 32 / nsl;
+  // consumer threads: up to 448 (plus producer and epilogue warps: 512 per
+  // CTA, 128 registers per thread), as many row phases as keep the stage
+  // ring at least three tiles deep
   const int tc_max = 448;
   int PH = nsl == 1 && Upad <= tc_max ? tc_max / Upad : 1;
-  auto ring_depth = [&](int ph) {
-    const long long tc = static_cast<long long>(Upad) * ph / nsl;
-    const long long rt = static_cast<long long>(RPT) * ph;
-    const long long red = 4 * ((rt * mr * (Upad / 32 / nsl) * 4 + 15) / 16 * 16);
-    const long long fixed = red + 64 + grp_bytes + 256;
-    const long long stage = RPT * nsl * tc * (4LL * bits + 8);
-    return (dev->smem_optin - fixed) / stage;
+  struct Sizes { long long w, s, red, stage; };
+  auto sizes = [&](int ph) {
+    Sizes z;
+    const long long rows = static_cast<long long>(RPT) * ph + RA - 1;
+    z.w = (rows * row_bytes + 15 + 15) / 16 * 16;
+    z.s = (rows * 2LL * G + 15 + 15) / 16 * 16;
+    z.red = (static_cast<long long>(RPT) * ph * mr * wpr * 4 + 15) / 16 * 16;
+    z.stage = z.w + 2 * z.s;
+    return z;
   };
-  while (PH > 1 && ring_depth(PH) < 3) --PH;
+  const int nred = 4;
+  auto depth_of = [&](int ph) {
+    const Sizes z = sizes(ph);
+    return (dev->smem_optin - grp_bytes - 256 - nred * (z.red + 16)) / (z.stage + 16);
+  };
+  while (PH > 1 && depth_of(PH) < 4) --PH;
   const int Tc = Upad * PH / nsl;
   if (Tc > tc_max || Tc % 32 != 0)
     return fail(QMV_ERR_UNSUPPORTED, "K=%d has no thread layout", K);
-  const int RT = RPT * PH;
-  const int wpr = Upad / 32 / nsl;
-  const int nred = 4;
-  const long long red_slot = (static_cast<long long>(RT) * mr * wpr * 4 + 15) / 16 * 16;
-  const long long bar_off = nred * red_slot;
-  const long long grp_off = (bar_off + 2 * nred * 8 + 15) / 16 * 16;
-  const long long cp_off = (grp_off + grp_bytes + 127) / 128 * 128;
-  // copy ring: depth stages of RPT rows x units x (unit bytes + scale/bias)
-  const long long stage = static_cast<long long>(RPT) * nsl * Tc * (4LL * bits + 8);
-  long long depth = (dev->smem_optin - cp_off) / stage;
-  if (depth > 4) depth = 4;
-  if (depth < 2)
+  const Sizes z = sizes(PH);
+  long long ns = depth_of(PH);
+  if (ns > 12) ns = 12;
+  if (ns < 2)
     return fail(QMV_ERR_UNSUPPORTED, "shape needs more shared memory than the device offers");
-  const long long smem = cp_off + depth * stage;
+  const int RT = RPT * PH;
   p.gs_shift = 0;
   while ((32 << p.gs_shift) < gs) ++p.gs_shift;
   p.G = G;
@@ -176,29 +180,39 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   p.Upad = Upad;
   p.PH = PH;
   p.RT = RT;
-  p.nred = nred;
+  p.RA = RA;
+  p.stages = static_cast<int>(ns);
   p.wpr = wpr;
   p.row_bytes = static_cast<uint32_t>(row_bytes);
   p.nch = p.mode == qmvk::MODE_GATHER ? 1 : (p.M + mr - 1) / mr;
-  p.red_off = 0;
-  p.red_slot = static_cast<uint32_t>(red_slot);
-  p.bar_off = static_cast<uint32_t>(bar_off);
-  p.grp_off = static_cast<uint32_t>(grp_off);
-  p.cp_off = static_cast<uint32_t>(cp_off);
-  p.depth = static_cast<int>(depth);
-  p.sb_pairs = (G % 2 == 0) ? 1 : 0;
-  pl.smem = static_cast<size_t>(smem);
+  p.w_stage = static_cast<uint32_t>(z.w);
+  p.s_stage = static_cast<uint32_t>(z.s);
+  const long long ring = ns * z.stage;
+  p.red_off = static_cast<uint32_t>((ring + (2 * ns + 2 * nred) * 8 + 15) / 16 * 16);
+  p.red_stage = static_cast<uint32_t>(z.red);
+  p.nred = nred;
+  p.grp_off = static_cast<uint32_t>(p.red_off + nred * z.red);
+  pl.smem = static_cast<size_t>(p.grp_off + grp_bytes);
   pl.mr = mr;
   pl.nsl = nsl;
-  pl.threads = Tc + 32;
-  // one CTA per SM; fewer when there is less work than SMs
-  long long work = p.mode == qmvk::MODE_GATHER
-                       ? static_cast<long long>(dev->sms)
-                       : static_cast<long long>(p.nmat) * p.nch * p.N;
-  if (work > 0x7fffffffLL)
-    return fail(QMV_ERR_UNSUPPORTED, "too many output rows in one call");
+  pl.threads = Tc + 64;
+  // One CTA per SM (fewer when there are fewer tiles).  Tiles are dealt
+  // round-robin, so the tile height is lowered until every CTA gets the
+  // same number of tiles to within one.
   long long grid = dev->sms;
-  if (work < grid) grid = work;
+  if (p.mode != qmvk::MODE_GATHER) {
+    const long long nseg = static_cast<long long>(p.nmat) * p.nch;
+    if (nseg * p.N > 0x7fffffffLL)
+      return fail(QMV_ERR_UNSUPPORTED, "too many output rows in one call");
+    const long long tiles = nseg * ((p.N + RT - 1) / RT);
+    if (tiles < grid) grid = tiles;
+    const long long per_cta = (tiles + grid - 1) / grid;
+    const long long tps_want = (per_cta * grid + nseg - 1) / nseg;
+    long long rte = (p.N + tps_want - 1) / tps_want;
+    if (rte < 1) rte = 1;
+    if (rte > RT) rte = RT;
+    p.RT = static_cast<int>(rte);
+  }
   pl.grid = static_cast<int>(grid < 1 ? 1 : grid);
   return QMV_OK;
 }
@@ -286,6 +300,7 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
   p.N = N;
   p.K = K;
   p.nmat = 1;
+  p.total_rows = N;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -325,6 +340,7 @@ int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
   p.N = N;
   p.K = K;
   p.nmat = 2;
+  p.total_rows = N;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -363,6 +379,7 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
   p.N = N;
   p.K = K;
   p.nmat = 1;
+  p.total_rows = N;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -420,6 +437,7 @@ int gather_qmv(const void *x, const uint32_t *w, const void *scales,
   p.num_pairs = num_pairs;
   p.num_x_rows = num_x_rows;
   p.num_experts = num_experts;
+  p.total_rows = static_cast<long long>(num_experts) * N;
   const int mr = num_pairs >= num_experts ? 2 : 1;
   if ((rc = make_plan(pl, bits, group_size, mr, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));

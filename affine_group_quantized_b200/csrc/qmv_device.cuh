@@ -281,17 +281,18 @@ __device__ __forceinline__ void prescale_unit(const float (&v)[32],
 // the odd nibbles of each word, masked; 2-bit: the four 2-bit lanes of each
 // byte, shifted and masked).  The activations of the unit are turned into
 // 22-bit fixed point relative to the unit's largest magnitude,
-// X_i = rint(x_i * 2^s) with |X_i| <= 2^22, and X_i is split into three
-// signed 8-bit digits: X = L2 * 2^16 + L1 * 2^8 + L0.  Every digit register
-// holds the digits of the four activations that meet the four codes of one
-// code register, so dp4a (four 8-bit products added to a 32-bit integer)
-// computes sum_i q_i * L_i exactly.  X_i equals x_i * 2^s exactly whenever
-// |x_i| is within 2^14 of the unit's largest |x| (a bf16 carries 8
-// significant bits); smaller elements are rounded to the unit's grid, an
-// error below 2^-23 of the unit's largest |x|.
+// X_i = rint(x_i * 2^s) with |X_i| <= 2^22, and the three low bytes of X_i's
+// two's-complement form are its digits: X = sext(b2) * 2^16 + b1 * 2^8 + b0
+// with b0, b1 unsigned.  Every digit register holds one digit of the four
+// activations that meet the four codes of one code register, so dp4a (four
+// 8-bit products added to a 32-bit integer) computes sum_i q_i * b_i exactly.
+// X_i equals x_i * 2^s exactly whenever |x_i| is within 2^14 of the unit's
+// largest |x| (a bf16 carries 8 significant bits); smaller elements are
+// rounded to the unit's grid, an error below 2^-23 of the unit's largest |x|.
 // Each digit sum starts from 0x4B400000, the bit pattern of 1.5 * 2^23: as
 // long as |sum| < 2^22 the 32-bit result read as a float is 1.5 * 2^23 + sum
-// exactly, so no integer-to-float conversion is needed.
+// exactly, so no integer-to-float conversion is needed; the same constant
+// rounds x * 2^s to an integer with one fused multiply-add.
 // ---------------------------------------------------------------------------
 
 template <int BITS>
@@ -309,8 +310,14 @@ __host__ __device__ constexpr int spread_reg(int bits, int i) {
 __host__ __device__ constexpr int spread_lane(int bits, int i) {
   return bits == 8 ? i % 4 : bits == 4 ? (i % 8) / 2 : (i % 16) / 4;
 }
+// code index held in byte lane `lane` of spread register r
+__host__ __device__ constexpr int spread_code(int bits, int r, int lane) {
+  return bits == 8 ? 4 * r + lane
+       : bits == 4 ? 8 * (r / 2) + (r % 2) + 2 * lane
+                   : 16 * (r / 4) + (r % 4) + 4 * lane;
+}
 
-// Spread register r (0..7) of a unit: four codes, one per byte.
+// Spread register R (0..7) of a unit: four codes, one per byte.
 template <int BITS, int R>
 __device__ __forceinline__ uint32_t spread_codes(const uint32_t (&wd)[BITS]) {
   if constexpr (BITS == 8) {
@@ -324,7 +331,14 @@ __device__ __forceinline__ uint32_t spread_codes(const uint32_t (&wd)[BITS]) {
   }
 }
 
-__device__ __forceinline__ int dp4a_su(int a, uint32_t b, int c) {
+// dp4a with unsigned (low digits) or signed (top digit) activation bytes;
+// the code bytes are unsigned.
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
   int d;
   asm("dp4a.s32.u32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
@@ -334,7 +348,7 @@ __device__ __forceinline__ int dp4a_su(int a, uint32_t b, int c) {
 // activation units (2^-s) and the plain activation sum times 2^s.
 template <int BITS>
 __device__ __forceinline__ void digits_unit(const float (&v)[32],
-                                            int (&dig)[3][8], float &inv,
+                                            uint32_t (&dig)[3][8], float &inv,
                                             float &vs) {
   float mx = 0.f, sum = 0.f;
 #pragma unroll
@@ -348,44 +362,46 @@ __device__ __forceinline__ void digits_unit(const float (&v)[32],
   const float sc = pow2i(s);
   inv = pow2i(-s);
   vs = sum * sc;
+  int X[32];
 #pragma unroll
-  for (int l = 0; l < 3; ++l)
+  for (int i = 0; i < 32; ++i)
+    X[i] = __float_as_int(fmaf(v[i], sc, kDigitBiasF)) - kDigitBias;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) dig[l][r] = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int X = __float2int_rn(v[i] * sc);
-    const int L0 = static_cast<int>(static_cast<int8_t>(X & 0xff));
-    const int X1 = (X - L0) >> 8;
-    const int L1 = static_cast<int>(static_cast<int8_t>(X1 & 0xff));
-    const int L2 = (X1 - L1) >> 8;
-    const int r = spread_reg(BITS, i), sh = 8 * spread_lane(BITS, i);
-    dig[0][r] |= (L0 & 0xff) << sh;
-    dig[1][r] |= (L1 & 0xff) << sh;
-    dig[2][r] |= (L2 & 0xff) << sh;
+  for (int r = 0; r < 8; ++r) {
+    const int a = X[spread_code(BITS, r, 0)], b = X[spread_code(BITS, r, 1)];
+    const int c = X[spread_code(BITS, r, 2)], d = X[spread_code(BITS, r, 3)];
+    const uint32_t ab = __byte_perm(a, b, 0x5140);  // a0 b0 a1 b1
+    const uint32_t cd = __byte_perm(c, d, 0x5140);  // c0 d0 c1 d1
+    dig[0][r] = __byte_perm(ab, cd, 0x5410);        // a0 b0 c0 d0
+    dig[1][r] = __byte_perm(ab, cd, 0x7632);        // a1 b1 c1 d1
+    const uint32_t ab2 = __byte_perm(a, b, 0x0062); // a2 b2
+    const uint32_t cd2 = __byte_perm(c, d, 0x0062); // c2 d2
+    dig[2][r] = __byte_perm(ab2, cd2, 0x5410);      // a2 b2 c2 d2
   }
 }
 
 template <int BITS, int MR, int R>
 __device__ __forceinline__ void dp_reg_2rows(const uint32_t (&w0)[BITS],
                                              const uint32_t (&w1)[BITS],
-                                             const int (&dig)[MR][3][8],
+                                             const uint32_t (&dig)[MR][3][8],
                                              int (&a0)[MR][3], int (&a1)[MR][3]) {
   const uint32_t b0 = spread_codes<BITS, R>(w0);
   const uint32_t b1 = spread_codes<BITS, R>(w1);
 #pragma unroll
-  for (int m = 0; m < MR; ++m)
-#pragma unroll
-    for (int l = 0; l < 3; ++l) {
-      a0[m][l] = dp4a_su(dig[m][l][R], b0, a0[m][l]);
-      a1[m][l] = dp4a_su(dig[m][l][R], b1, a1[m][l]);
-    }
+  for (int m = 0; m < MR; ++m) {
+    a0[m][0] = dp4a_uu(dig[m][0][R], b0, a0[m][0]);
+    a0[m][1] = dp4a_uu(dig[m][1][R], b0, a0[m][1]);
+    a0[m][2] = dp4a_su(dig[m][2][R], b0, a0[m][2]);
+    a1[m][0] = dp4a_uu(dig[m][0][R], b1, a1[m][0]);
+    a1[m][1] = dp4a_uu(dig[m][1][R], b1, a1[m][1]);
+    a1[m][2] = dp4a_su(dig[m][2][R], b1, a1[m][2]);
+  }
 }
 
 template <int BITS, int MR, int... R>
 __device__ __forceinline__ void unit_dp_2rows_impl(
     const uint32_t (&w0)[BITS], const uint32_t (&w1)[BITS],
-    const int (&dig)[MR][3][8], int (&a0)[MR][3], int (&a1)[MR][3],
+    const uint32_t (&dig)[MR][3][8], int (&a0)[MR][3], int (&a1)[MR][3],
     std::integer_sequence<int, R...>) {
   (dp_reg_2rows<BITS, MR, R>(w0, w1, dig, a0, a1), ...);
 }
@@ -395,7 +411,7 @@ __device__ __forceinline__ void unit_dp_2rows_impl(
 template <int BITS, int MR>
 __device__ __forceinline__ void unit_dp_2rows(const uint32_t (&w0)[BITS],
                                               const uint32_t (&w1)[BITS],
-                                              const int (&dig)[MR][3][8],
+                                              const uint32_t (&dig)[MR][3][8],
                                               float (&r0)[MR], float (&r1)[MR]) {
   int a0[MR][3], a1[MR][3];
 #pragma unroll

@@ -1,20 +1,23 @@
 // qmv_stream.cuh -- the persistent weight-streaming GEMV kernel (CUDA cores).
 //
-// One CTA per SM with two warp roles:
+// One CTA per SM with three warp roles:
+//   * producer warp: streams tiles of packed weight rows, with their scales
+//     and biases, from HBM into a ring of shared-memory stages.  The 32 lanes
+//     copy each tile's contiguous byte ranges with 16-byte cp.async (a warp
+//     instruction moves 512 contiguous bytes); each lane's copies complete on
+//     the stage's mbarrier (cp.async.mbarrier.arrive.noinc).
 //   * consumer warps: each thread owns one 32-code "unit" column of the
-//     weight rows and a row phase.  It streams its unit of its rows from HBM
-//     with asynchronous 16-byte copies (cp.async) into its own slots of a
-//     shared-memory ring several tiles deep; a warp's copies of one row are
-//     32 consecutive units (one contiguous 512-byte span at 4 bits).  Each
-//     thread reads back only what it copied itself, so no barrier is needed
-//     between copy and use: cp.async.wait_group per thread.  Codes are decoded in registers and multiplied with the unit's
+//     weight rows (its activations stay in registers) and a row phase.  It
+//     decodes its unit of its rows of the stage, multiplies with the
 //     activations (8-bit integer dot products for 2/4/8-bit codes, fp32 FMAs
-//     for 3/5/6-bit codes), the group scale and bias are applied, and the warp
-//     reduces the row partials with shuffles into a small shared ring;
-//   * one epilogue warp: adds the per-warp partials of each output in a fixed
+//     for 3/5/6-bit codes), applies the group scale and bias, and the warp
+//     reduces the row partials with shuffles into the stage's partial-sum
+//     buffer;
+//   * epilogue warp: adds the per-warp partials of each output in a fixed
 //     order, adds the residual if any, rounds once to bf16 and stores.
-// Consumers and the epilogue hand ring slots over with mbarriers; consumer
-// warps never wait for each other.
+// Stage handoffs are mbarrier phases; consumer warps never wait for each
+// other.  Tiles are dealt to CTAs round-robin, so that at any moment all SMs
+// stream from one compact window of memory.
 //
 // The same kernel serves every entry point through `mode`:
 //   MODE_QMV      y = x @ dequant(W).T
@@ -25,8 +28,8 @@
 //                 routed to it
 //
 // Work is a list of "segments", each one weight matrix (or expert) paired
-// with up to MR activation rows; a segment's N rows are cut into tiles of
-// RT rows.  Each CTA owns a contiguous range of the (segment, row) space.
+// with up to MR activation rows; a segment's N rows are cut into tiles of at
+// most RT rows.
 #pragma once
 
 #include "qmv_device.cuh"
@@ -53,26 +56,27 @@ struct StreamParams {
   int gs_shift;           // log2(group_size / 32): unit -> group
   int U, Upad;            // units per row (K/32) and padded count (>= 32)
   int PH;                 // row phases: Upad threads per row, PH rows at once
-  int RT;                 // rows per tile = RPT * PH (RPT fixed per kernel)
+  int RT;                 // rows per tile (at most RPT * PH)
+  int RA;                 // row alignment making copy starts 16-byte aligned
   int nmat;               // weight matrices (1, or 2 for gate/up)
   int nch;                // activation chunks per matrix: ceil(M / MR)
-  int nred;               // slots in the partial-sum ring
+  int stages;             // depth of the stage ring
   int wpr;                // partial-sum slots per row (consumer warps per row)
   uint32_t row_bytes;     // K * bits / 8
+  long long total_rows;   // rows in each weight array (N, or E*N)
   int num_pairs, num_x_rows, num_experts;
-  uint32_t red_off;       // smem offset of the partial-sum ring
-  uint32_t red_slot;      // bytes of one ring slot
-  uint32_t bar_off;       // smem offset of the ring's mbarriers
-  uint32_t grp_off;       // smem offset of the gather grouping tables
-  uint32_t cp_off;        // smem offset of the copy ring
-  int depth;              // tiles in the copy ring
-  int sb_pairs;           // scales/biases copied as aligned 4-byte pairs (G even)
+  uint32_t w_stage, s_stage;  // bytes of the W and of the S (= B) region
+  uint32_t red_off;           // smem offset of the partial-sum ring
+  uint32_t red_stage;         // bytes of one partial-sum ring slot
+  int nred;                   // slots in the partial-sum ring
+  uint32_t grp_off;           // smem offset of the gather grouping tables
 };
 
 // ---------------------------------------------------------------------------
-// Tiles and the stage ring, walked with incremental 32-bit bookkeeping.
-// Producer, consumers and epilogue run the same walk, so they agree on every
-// tile without communicating.
+// Tiles.  A segment has tps = ceil(N / RT) tiles; the tiles of all segments
+// are numbered segment by segment and dealt round-robin: CTA c gets tiles
+// c, c + G, c + 2G, ...  Every role of a CTA runs the same walk and uses the
+// tile's position in it as its stage index.
 // ---------------------------------------------------------------------------
 struct Tile {
   int seg;    // segment index
@@ -81,37 +85,35 @@ struct Tile {
 };
 
 struct TileWalker {
-  int seg, row, left, N, RT;
+  int seg, tj, tps, nseg, step, N, RT;
   int stages, st;
   uint32_t phase;
 
-  __device__ __forceinline__ void init(long long v0, long long v1, int N_,
-                                       int RT_, int stages_) {
+  __device__ __forceinline__ void init(int nseg_, int N_, int RT_, int stages_) {
     N = N_;
     RT = RT_;
+    nseg = nseg_;
     stages = stages_;
-    seg = static_cast<int>(v0 / N);
-    row = static_cast<int>(v0 - static_cast<long long>(seg) * N);
-    left = static_cast<int>(v1 - v0);
+    tps = (N + RT - 1) / RT;
+    step = gridDim.x;
+    seg = blockIdx.x / tps;
+    tj = blockIdx.x - seg * tps;
     st = 0;
     phase = 0;
   }
   __device__ __forceinline__ bool next(Tile &t) {
-    if (left <= 0) return false;
-    int n = RT < N - row ? RT : N - row;
-    n = n < left ? n : left;
+    if (seg >= nseg) return false;
     t.seg = seg;
-    t.row = row;
-    t.nrows = n;
-    row += n;
-    left -= n;
-    if (row == N) {
-      row = 0;
+    t.row = tj * RT;
+    t.nrows = N - t.row < RT ? N - t.row : RT;
+    tj += step;
+    while (tj >= tps) {
+      tj -= tps;
       ++seg;
     }
     return true;
   }
-  __device__ __forceinline__ void advance_slot() {
+  __device__ __forceinline__ void advance_stage() {
     if (++st == stages) {
       st = 0;
       phase ^= 1u;
@@ -277,26 +279,155 @@ __device__ __forceinline__ long long abs_row(const StreamParams &p, int arr,
 }
 
 // ---------------------------------------------------------------------------
+// Shared-memory helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed;
+// the arrival counts towards the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// One unit (4*BITS bytes, starting at a multiple of 4*BITS) from shared
+// memory with the widest aligned loads.
+template <int BITS>
+__device__ __forceinline__ void lds_unit(uint32_t a, uint32_t (&wd)[BITS]) {
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS / 4; ++i) {
+      const uint4 v = lds128(a + 16 * i);
+      wd[4 * i] = v.x; wd[4 * i + 1] = v.y; wd[4 * i + 2] = v.z; wd[4 * i + 3] = v.w;
+    }
+  } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS / 2; ++i) {
+      const uint2 v = lds64(a + 8 * i);
+      wd[2 * i] = v.x; wd[2 * i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) wd[i] = lds32(a + 4 * i);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Producer warp: copies byte range [begin, end) of an array into shared
+// memory at `dst` (begin 16-byte aligned), 16 bytes per lane per step.  The
+// last partial 16 bytes, if the array ends there, are copied in 4-byte pieces
+// (elem = 4) or by lane 0 with plain loads and stores (elem = 2).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void warp_copy(uint32_t dst, const uint8_t *base,
+                                          long long begin, long long end,
+                                          long long total, int elem, int lane,
+                                          bool &plain) {
+  long long e16 = (end + 15) & ~15LL;
+  if (e16 > total) e16 = end & ~15LL;
+  for (long long o = begin + 16LL * lane; o < e16; o += 512)
+    cp_async16(dst + static_cast<uint32_t>(o - begin), base + o);
+  for (long long o = (e16 > begin ? e16 : begin) + 4LL * lane; o + 4 <= end;
+       o += 128)
+    if (elem == 4) cp_async4(dst + static_cast<uint32_t>(o - begin), base + o);
+  if (elem == 2 && lane == 0) {
+    for (long long o = e16 > begin ? e16 : begin; o < end; o += 2) {
+      const uint16_t v = *reinterpret_cast<const uint16_t *>(base + o);
+      asm volatile("st.shared.u16 [%0], %1;\n" ::"r"(dst + static_cast<uint32_t>(o - begin)),
+                   "h"(v)
+                   : "memory");
+      plain = true;
+    }
+  }
+}
+
+template <int MR>
+__device__ void producer_loop(const StreamParams &p, unsigned char *smem,
+                              uint64_t *full, uint64_t *empty, const Groups &g,
+                              int nseg, int lane) {
+  TileWalker tw;
+  tw.init(nseg, p.N, p.RT, p.stages);
+  Tile t;
+  const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
+  const uint32_t base = smem_u32(smem);
+  while (tw.next(t)) {
+    const int st = tw.st;
+    if (!mbar_wait(&empty[st], tw.phase ^ 1u)) {
+      if (p.err && lane == 0) atomicOr(p.err, 2);
+      return;
+    }
+    const Seg sg = seg_info<MR>(p, g, t.seg);
+    const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
+    const long long ar = abs_row(p, sg.arr, t.row);
+    const int lead = static_cast<int>(ar & (p.RA - 1));  // RA: power of two
+    const long long r0 = ar - lead, r1 = ar + t.nrows;
+    const uint32_t dst = base + st * stage_bytes;
+    const long long sb = 2LL * p.G;
+    bool plain = false;
+    warp_copy(dst, p.w[w_arr], r0 * p.row_bytes, r1 * p.row_bytes,
+              p.total_rows * p.row_bytes, 4, lane, plain);
+    warp_copy(dst + p.w_stage, reinterpret_cast<const uint8_t *>(p.s[w_arr]),
+              r0 * sb, r1 * sb, p.total_rows * sb, 2, lane, plain);
+    warp_copy(dst + p.w_stage + p.s_stage,
+              reinterpret_cast<const uint8_t *>(p.b[w_arr]), r0 * sb, r1 * sb,
+              p.total_rows * sb, 2, lane, plain);
+    // every lane's copies arrive asynchronously; lane 0 also arrives once
+    // for its plain stores (if any), keeping the expected count fixed
+    cp_async_arrive(&full[st]);
+    if (lane == 0) mbar_arrive(&full[st]);
+    tw.advance_stage();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Epilogue warp: sums the consumer warps' partials of each output in a fixed
-// order, adds the residual, rounds once to bf16 and stores.
+// order, adds the residual, rounds once to bf16 and stores; then releases the
+// partial-sum slot.
 // ---------------------------------------------------------------------------
 template <int MR>
 __device__ void epilogue_loop(const StreamParams &p, unsigned char *smem,
                               uint64_t *redfull, uint64_t *redempty,
-                              const Groups &g, long long v0, long long v1,
-                              int lane) {
+                              const Groups &g, int nseg, int lane) {
   TileWalker tw;
-  tw.init(v0, v1, p.N, p.RT, p.nred);
+  tw.init(nseg, p.N, p.RT, p.nred);
   Tile t;
   while (tw.next(t)) {
     const int st = tw.st;
     if (!mbar_wait(&redfull[st], tw.phase)) {
-      if (p.err) atomicOr(p.err, 2);
+      if (p.err && lane == 0) atomicOr(p.err, 2);
       return;
     }
     const Seg sg = seg_info<MR>(p, g, t.seg);
     const float *rb =
-        reinterpret_cast<const float *>(smem + p.red_off + st * p.red_slot);
+        reinterpret_cast<const float *>(smem + p.red_off + st * p.red_stage);
     for (int o = lane; o < t.nrows * MR; o += 32) {
       const int r = o / MR, m = o % MR;
       if (m < sg.count) {
@@ -315,136 +446,13 @@ __device__ void epilogue_loop(const StreamParams &p, unsigned char *smem,
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&redempty[st]);
-    tw.advance_slot();
+    tw.advance_stage();
   }
 }
 
 // ---------------------------------------------------------------------------
 // Consumers
 // ---------------------------------------------------------------------------
-
-// Asynchronous global -> shared copies of 16, 8 or 4 bytes (cp.async).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(a));
-  return v;
-}
-
-// Layout of one thread's copy of one row in the ring: the unit's bytes in
-// "planes" of 16, 8 or 4 bytes (the largest that divides the unit), each
-// plane of all consumer threads contiguous, so that the reads of a warp hit
-// 32 consecutive 16/8/4-byte slots (no bank conflicts); then the scale and
-// the bias, each as the aligned 4-byte pair that holds it (or the value
-// itself when the pairs are not 4-byte aligned).
-template <int BITS>
-struct CopyLayout {
-  static constexpr int kUnitBytes = 4 * BITS;
-  static constexpr int kPlane = BITS % 4 == 0 ? 16 : (BITS % 2 == 0 ? 8 : 4);
-  static constexpr int kPlanes = kUnitBytes / kPlane;
-  // bytes of one row of the ring for Tc threads
-  static __host__ __device__ constexpr uint32_t row_bytes(int tc) {
-    return static_cast<uint32_t>(tc) * (kUnitBytes + 8);
-  }
-};
-
-// Issue the copies of the thread's rows of one tile into ring stage `stage`.
-template <int BITS, int RPT>
-__device__ __forceinline__ void issue_tile(const StreamParams &p, const Tile &t,
-                                           int arr, int w_arr, int ph, int u,
-                                           int tid, int Tc, uint32_t stage_base) {
-  using CL = CopyLayout<BITS>;
-  const long long r0 = abs_row(p, arr, t.row);
-  const uint8_t *wb = p.w[w_arr] + static_cast<size_t>(u) * CL::kUnitBytes;
-  const int grp = u >> p.gs_shift;
-  const uint32_t rowb = CL::row_bytes(Tc);
-#pragma unroll
-  for (int rr = 0; rr < RPT; ++rr) {
-    const int r = ph + rr * p.PH;
-    if (r < t.nrows) {
-      const long long row = r0 + r;
-      const uint8_t *src = wb + row * p.row_bytes;
-      const uint32_t dst = stage_base + rr * rowb;
-#pragma unroll
-      for (int c = 0; c < CL::kPlanes; ++c) {
-        const uint32_t d = dst + (c * Tc + tid) * CL::kPlane;
-        if constexpr (CL::kPlane == 16) cp_async16(d, src + 16 * c);
-        else if constexpr (CL::kPlane == 8) cp_async8(d, src + 8 * c);
-        else cp_async4(d, src + 4 * c);
-      }
-      const long long si = row * p.G + grp;
-      const uint32_t dsb = dst + Tc * CL::kUnitBytes + tid * 8;
-      if (p.sb_pairs) {
-        cp_async4(dsb, p.s[w_arr] + (si & ~1LL));
-        cp_async4(dsb + 4, p.b[w_arr] + (si & ~1LL));
-      }
-    }
-  }
-}
-
-// Read back one row of the thread's unit from ring stage `stage_base`.
-template <int BITS>
-__device__ __forceinline__ void read_row(const StreamParams &p, uint32_t stage_base,
-                                         int rr, int tid, int Tc, int grp_odd,
-                                         long long row, int w_arr, int grp,
-                                         uint32_t (&w)[BITS], uint32_t &sb) {
-  using CL = CopyLayout<BITS>;
-  const uint32_t dst = stage_base + rr * CL::row_bytes(Tc);
-#pragma unroll
-  for (int c = 0; c < CL::kPlanes; ++c) {
-    const uint32_t a = dst + (c * Tc + tid) * CL::kPlane;
-    if constexpr (CL::kPlane == 16) {
-      const uint4 v = lds128(a);
-      w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-    } else if constexpr (CL::kPlane == 8) {
-      const uint2 v = lds64(a);
-      w[2 * c] = v.x; w[2 * c + 1] = v.y;
-    } else {
-      w[c] = lds32(a);
-    }
-  }
-  if (p.sb_pairs) {
-    const uint2 v = lds64(dst + Tc * CL::kUnitBytes + tid * 8);
-    // the wanted bf16 is the low half for an even group index, else the high
-    const uint32_t s = grp_odd ? (v.x >> 16) : (v.x & 0xffffu);
-    const uint32_t b = grp_odd ? (v.y & 0xffff0000u) : (v.y << 16);
-    sb = s | b;
-  } else {
-    const long long si = row * p.G + grp;
-    sb = static_cast<uint32_t>(__ldg(p.s[w_arr] + si)) |
-         (static_cast<uint32_t>(__ldg(p.b[w_arr] + si)) << 16);
-  }
-}
 
 // Transposed butterfly over the 32 lanes of a warp: NV partial sums per lane
 // in; afterwards lane l holds the full sum of value l / (32 / NV) in vals[0].
@@ -509,7 +517,7 @@ __device__ __forceinline__ void unit_activations(const StreamParams &p, int u,
 template <int BITS, int MR>
 struct UnitActs {
   static constexpr bool kInt = kIntPath<BITS>;
-  int dig[kInt ? MR : 1][3][8];
+  uint32_t dig[kInt ? MR : 1][3][8];
   float2 xp[kInt ? 1 : MR][16];
   float back[MR], vs[MR];
 
@@ -579,38 +587,47 @@ __device__ __forceinline__ void row_pair_dot(const uint32_t (&w0)[BITS],
 // BITS: code width; MR: activation rows per segment (1 or 2); NSL: units per
 // consumer thread (1 or 2).
 template <int BITS, int MR, int NSL>
-__global__ void __launch_bounds__(480, 1)
+__global__ void __launch_bounds__(512, 1)
     qmv_stream_kernel(const StreamParams p) {
   constexpr int RPT = rows_per_thread<BITS, MR, NSL>();
-  using CL = CopyLayout<BITS>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
   const int Tc = p.Upad * p.PH / NSL;  // consumer threads
-  uint64_t *redfull = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+  const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
+  uint64_t *full = reinterpret_cast<uint64_t *>(
+      smem + static_cast<size_t>(p.stages) * stage_bytes);
+  uint64_t *empty = full + p.stages;
+  uint64_t *redfull = empty + p.stages;
   uint64_t *redempty = redfull + p.nred;
 
   if (tid == 0) {
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(&full[i], 33);      // 32 async arrivals + lane 0
+      mbar_init(&empty[i], Tc / 32);  // consumer warps
+    }
     for (int i = 0; i < p.nred; ++i) {
       mbar_init(&redfull[i], Tc / 32);
-      mbar_init(&redempty[i], 1);
+      mbar_init(&redempty[i], 1);   // epilogue warp
     }
     fence_mbar_init();
   }
   Groups g{};
-  long long V;
+  int nseg;
   if (p.mode == MODE_GATHER) {
     g = groups_at(smem, p);
     build_groups<MR>(p, g, tid, blockDim.x);  // ends with __syncthreads
-    V = static_cast<long long>(*g.nseg) * p.N;
+    nseg = *g.nseg;
   } else {
     __syncthreads();
-    V = static_cast<long long>(p.nmat) * p.nch * p.N;
+    nseg = p.nmat * p.nch;
   }
-  const long long v0 = V * blockIdx.x / gridDim.x;
-  const long long v1 = V * (blockIdx.x + 1) / gridDim.x;
 
   if (tid >= Tc) {
-    epilogue_loop<MR>(p, smem, redfull, redempty, g, v0, v1, tid - Tc);
+    const int lane = tid & 31;
+    if (tid < Tc + 32)
+      producer_loop<MR>(p, smem, full, empty, g, nseg, lane);
+    else
+      epilogue_loop<MR>(p, smem, redfull, redempty, g, nseg, lane);
     return;
   }
 
@@ -621,37 +638,26 @@ __global__ void __launch_bounds__(480, 1)
   for (int j = 0; j < NSL; ++j) su[j] = (tid + j * Tc) % p.Upad;
   const int ph = tid / p.Upad;  // NSL == 2 implies PH == 1 and ph == 0
   const int wslot = su[0] / 32;
-  const uint32_t ring = smem_u32(smem) + p.cp_off;
-  // one stage = RPT rows for every consumer thread and every slot
-  const uint32_t stage_bytes = RPT * NSL * CL::row_bytes(Tc);
-
-  // prefetch: the first depth-1 tiles
-  TileWalker tw_issue;
-  tw_issue.init(v0, v1, p.N, p.RT, p.depth);
-  auto issue_next = [&](int stage) {
-    Tile ti;
-    if (tw_issue.next(ti)) {
-      const Seg si = seg_info<MR>(p, g, ti.seg);
-      const int w_arr = p.mode == MODE_GATHER ? 0 : si.arr;
-#pragma unroll
-      for (int j = 0; j < NSL; ++j)
-        if (su[j] < p.U)
-          issue_tile<BITS, RPT>(p, ti, si.arr, w_arr, ph, su[j], tid, Tc,
-                                ring + stage * stage_bytes +
-                                    j * RPT * CL::row_bytes(Tc));
-    }
-    cp_async_commit();  // possibly empty: keeps the group count regular
+  const uint32_t row_bytes = p.row_bytes;
+  const uint32_t srow_bytes = 2u * p.G;
+  const uint32_t rstep = row_bytes * p.PH, sstep = srow_bytes * p.PH;
+  const uint32_t smem_base = smem_u32(smem);
+  // rows of the thread inside a tile of n rows (warp-uniform)
+  auto rows_of = [&](int n) {
+    return n > ph ? min(RPT, (n - ph + p.PH - 1) / p.PH) : 0;
   };
-  for (int k = 0; k < p.depth - 1; ++k) issue_next(k);
+  const int nfull = rows_of(p.RT);
 
   UnitActs<BITS, MR> ua[NSL];
   int loaded = -1;  // key of the activation rows held in ua
 
-  TileWalker tw;
-  tw.init(v0, v1, p.N, p.RT, p.nred);
-  Tile t;
-  int cstage = 0;
+  TileWalker tw, twr;  // stage ring and partial-sum ring positions
+  tw.init(nseg, p.N, p.RT, p.stages);
+  twr.init(nseg, p.N, p.RT, p.nred);
+  Tile t, tr;
   while (tw.next(t)) {
+    twr.next(tr);
+    const int st = tw.st;
     const Seg sg = seg_info<MR>(p, g, t.seg);
     if (sg.key != loaded) {
       int xr[MR];
@@ -661,19 +667,17 @@ __global__ void __launch_bounds__(480, 1)
       for (int j = 0; j < NSL; ++j) ua[j].load(p, su[j], xr);
       loaded = sg.key;
     }
-    // keep depth-1 tiles in flight: issue the tile depth-1 ahead, then wait
-    // until this tile's copies have landed
-    int istage = cstage + p.depth - 1;
-    if (istage >= p.depth) istage -= p.depth;
-    issue_next(istage);
-    switch (p.depth) {  // at most depth-1 newer groups may stay in flight
-      case 2: cp_async_wait<1>(); break;
-      case 3: cp_async_wait<2>(); break;
-      default: cp_async_wait<3>(); break;
+    const long long ar = abs_row(p, sg.arr, t.row);
+    const uint32_t lead = static_cast<uint32_t>(ar & (p.RA - 1));
+    const int nvalid = t.nrows == p.RT ? nfull : rows_of(t.nrows);
+
+    if (!mbar_wait(&full[st], tw.phase)) {
+      if (p.err && lane == 0) atomicOr(p.err, 2);
+      return;
     }
-    const long long r0 = abs_row(p, sg.arr, t.row);
-    const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
-    const int nvalid = t.nrows > ph ? min(RPT, (t.nrows - ph + p.PH - 1) / p.PH) : 0;
+    const uint32_t wst = smem_base + st * stage_bytes + (lead + ph) * row_bytes;
+    const uint32_t sst =
+        smem_base + st * stage_bytes + p.w_stage + (lead + ph) * srow_bytes;
 
     float part[RPT * MR];
 #pragma unroll
@@ -682,21 +686,22 @@ __global__ void __launch_bounds__(480, 1)
     for (int j = 0; j < NSL; ++j) {
       const int u = su[j];
       if (u < p.U) {
-        const int grp = u >> p.gs_shift;
-        const uint32_t sbase = ring + cstage * stage_bytes + j * RPT * CL::row_bytes(Tc);
         float pj[RPT * MR];
 #pragma unroll
         for (int i = 0; i < RPT * MR; ++i) pj[i] = 0.f;
+        const uint32_t aw = wst + static_cast<uint32_t>(u) * (4 * BITS);
+        const uint32_t as = sst + 2u * static_cast<uint32_t>(u >> p.gs_shift);
 #pragma unroll
         for (int q = 0; q < RPT / 2; ++q) {
           if (2 * q < nvalid) {  // warp-uniform
-            uint32_t w0[BITS], w1[BITS], sb0, sb1;
-            // a row past the tile end reads the first row's data again
-            const int rb1 = 2 * q + 1 < nvalid ? 2 * q + 1 : 2 * q;
-            read_row<BITS>(p, sbase, 2 * q, tid, Tc, grp & 1,
-                           r0 + ph + 2 * q * p.PH, w_arr, grp, w0, sb0);
-            read_row<BITS>(p, sbase, rb1, tid, Tc, grp & 1,
-                           r0 + ph + rb1 * p.PH, w_arr, grp, w1, sb1);
+            // a row past the tile end reuses the pair's first row
+            const int rb = 2 * q + 1 < nvalid ? 2 * q + 1 : 2 * q;
+            uint32_t w0[BITS], w1[BITS];
+            lds_unit<BITS>(aw + 2 * q * rstep, w0);
+            lds_unit<BITS>(aw + rb * rstep, w1);
+            const uint32_t sa = as + 2 * q * sstep, sb = as + rb * sstep;
+            const uint32_t sb0 = lds16(sa) | (lds16(sa + p.s_stage) << 16);
+            const uint32_t sb1 = lds16(sb) | (lds16(sb + p.s_stage) << 16);
             row_pair_dot<BITS, MR>(w0, sb0, w1, sb1, ua[j], pj + (2 * q) * MR,
                                    pj + (2 * q + 1) * MR);
           }
@@ -706,17 +711,19 @@ __global__ void __launch_bounds__(480, 1)
           part[i] = fmaf(pj[i], ua[j].back[i % MR], part[i]);
       }
     }
-    if (++cstage == p.depth) cstage = 0;
+    // done reading the stage's weights, scales and biases
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
 
     // ---- reduce over the warp's units; one partial per row and x row ----
-    const int st = tw.st;
     constexpr int NV = RPT * MR;
     transpose_reduce<NV>(part, lane);
-    if (!mbar_wait(&redempty[st], tw.phase ^ 1u)) {
-      if (p.err) atomicOr(p.err, 2);
+    const int rs = twr.st;
+    if (!mbar_wait(&redempty[rs], twr.phase ^ 1u)) {
+      if (p.err && lane == 0) atomicOr(p.err, 2);
       return;
     }
-    float *rbuf = reinterpret_cast<float *>(smem + p.red_off + st * p.red_slot);
+    float *rbuf = reinterpret_cast<float *>(smem + p.red_off + rs * p.red_stage);
     if ((lane % (32 / NV)) == 0) {
       const int idx = lane / (32 / NV);
       const int rr = idx / MR, m = idx % MR;
@@ -724,10 +731,10 @@ __global__ void __launch_bounds__(480, 1)
       if (r < t.nrows) rbuf[(r * MR + m) * p.wpr + wslot] = part[0];
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&redfull[st]);
-    tw.advance_slot();
+    if (lane == 0) mbar_arrive(&redfull[rs]);
+    tw.advance_stage();
+    twr.advance_stage();
   }
-  cp_async_wait<0>();  // nothing may be in flight when the thread exits
 }
 
 }  // namespace qmvk
