@@ -159,9 +159,13 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
     return z;
   };
   const int nred = 4;
+  // sub-stages (one per row pair of the consumer threads) need every row
+  // start 16-byte aligned
+  const int nsub = (RA == 1 && RPT >= 4) ? RPT / 2 : 1;
   auto depth_of = [&](int ph) {
     const Sizes z = sizes(ph);
-    return (dev->smem_optin - grp_bytes - 256 - nred * (z.red + 16)) / (z.stage + 16);
+    return (dev->smem_optin - grp_bytes - 256 - nred * (z.red + 16)) /
+           (z.stage + 8 * (nsub + 1));
   };
   while (PH > 1 && depth_of(PH) < 4) --PH;
   const int Tc = Upad * PH / nsl;
@@ -182,13 +186,15 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   p.RT = RT;
   p.RA = RA;
   p.stages = static_cast<int>(ns);
+  p.nsub = nsub;
   p.wpr = wpr;
   p.row_bytes = static_cast<uint32_t>(row_bytes);
   p.nch = p.mode == qmvk::MODE_GATHER ? 1 : (p.M + mr - 1) / mr;
   p.w_stage = static_cast<uint32_t>(z.w);
   p.s_stage = static_cast<uint32_t>(z.s);
   const long long ring = ns * z.stage;
-  p.red_off = static_cast<uint32_t>((ring + (2 * ns + 2 * nred) * 8 + 15) / 16 * 16);
+  p.red_off = static_cast<uint32_t>(
+      (ring + ((nsub + 1) * ns + 2 * nred) * 8 + 15) / 16 * 16);
   p.red_stage = static_cast<uint32_t>(z.red);
   p.nred = nred;
   p.grp_off = static_cast<uint32_t>(p.red_off + nred * z.red);
@@ -217,18 +223,18 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   return QMV_OK;
 }
 
-template <int BITS, int MR, int NSL>
+template <int BITS, int MR, int NSL, bool SILU>
 int &granted_smem(int dev) {
   static int granted[kMaxDevices] = {};
   return granted[dev];
 }
 
-template <int BITS, int MR, int NSL>
+template <int BITS, int MR, int NSL, bool SILU>
 int launch_t(const Plan &pl, cudaStream_t stream) {
-  auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL>;
+  auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL, SILU>;
   int dev = 0;
   cudaGetDevice(&dev);
-  int &granted = granted_smem<BITS, MR, NSL>(dev);
+  int &granted = granted_smem<BITS, MR, NSL, SILU>(dev);
   if (static_cast<int>(pl.smem) > granted) {
     cudaError_t e = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -245,11 +251,17 @@ int launch_t(const Plan &pl, cudaStream_t stream) {
   return ok();
 }
 
+template <int BITS, bool SILU>
+int launch_shape(const Plan &pl, cudaStream_t stream) {
+  if (pl.nsl == 2) return launch_t<BITS, 1, 2, SILU>(pl, stream);
+  if (pl.mr == 2) return launch_t<BITS, 2, 1, SILU>(pl, stream);
+  return launch_t<BITS, 1, 1, SILU>(pl, stream);
+}
+
 template <int BITS>
 int launch_bits(const Plan &pl, cudaStream_t stream) {
-  if (pl.nsl == 2) return launch_t<BITS, 1, 2>(pl, stream);
-  if (pl.mr == 2) return launch_t<BITS, 2, 1>(pl, stream);
-  return launch_t<BITS, 1, 1>(pl, stream);
+  if (pl.p.mode == qmvk::MODE_SILU) return launch_shape<BITS, true>(pl, stream);
+  return launch_shape<BITS, false>(pl, stream);
 }
 
 int launch(const Plan &pl, int bits, cudaStream_t stream) {

@@ -83,9 +83,13 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src,
       : "memory");
 }
 
-// Named barrier over the first `nthreads` threads (a multiple of 32).
+// Named barrier `id` over `nthreads` threads (a multiple of 32): wait for
+// all of them, or only signal arrival without waiting.
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------------------

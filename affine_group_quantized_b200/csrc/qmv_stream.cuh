@@ -1,11 +1,11 @@
 // qmv_stream.cuh -- the persistent weight-streaming GEMV kernel (CUDA cores).
 //
 // One CTA per SM with three warp roles:
-//   * producer warp: streams tiles of packed weight rows, with their scales
-//     and biases, from HBM into a ring of shared-memory stages.  The 32 lanes
-//     copy each tile's contiguous byte ranges with 16-byte cp.async (a warp
-//     instruction moves 512 contiguous bytes); each lane's copies complete on
-//     the stage's mbarrier (cp.async.mbarrier.arrive.noinc).
+//   * producer warp: one thread streams tiles of packed weight rows, with
+//     their scales and biases, from HBM into a ring of shared-memory stages
+//     with 1-D bulk copies (a tile is three contiguous byte ranges) that
+//     complete on the stage's mbarrier.  It sets up the barriers itself and
+//     starts the first stages before the other warps are released.
 //   * consumer warps: each thread owns one 32-code "unit" column of the
 //     weight rows (its activations stay in registers) and a row phase.  It
 //     decodes its unit of its rows of the stage, multiplies with the
@@ -61,6 +61,7 @@ struct StreamParams {
   int nmat;               // weight matrices (1, or 2 for gate/up)
   int nch;                // activation chunks per matrix: ceil(M / MR)
   int stages;             // depth of the stage ring
+  int nsub;               // sub-stages per stage (1, or rows-per-thread / 2)
   int wpr;                // partial-sum slots per row (consumer warps per row)
   uint32_t row_bytes;     // K * bits / 8
   long long total_rows;   // rows in each weight array (N, or E*N)
@@ -151,7 +152,7 @@ __device__ __forceinline__ Groups groups_at(unsigned char *smem,
 }
 
 template <int MR>
-__device__ void build_groups(const StreamParams &p, Groups g, int tid,
+__device__ __forceinline__ void build_groups(const StreamParams &p, Groups g, int tid,
                              int nthreads) {
   const int E = p.num_experts, P = p.num_pairs;
   for (int e = tid; e < E; e += nthreads) g.cnt[e] = 0;
@@ -281,21 +282,6 @@ __device__ __forceinline__ long long abs_row(const StreamParams &p, int arr,
 // ---------------------------------------------------------------------------
 // Shared-memory helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src)
-               : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed;
-// the arrival counts towards the barrier's expected count.
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
@@ -342,69 +328,132 @@ __device__ __forceinline__ void lds_unit(uint32_t a, uint32_t (&wd)[BITS]) {
 }
 
 // ---------------------------------------------------------------------------
-// Producer warp: copies byte range [begin, end) of an array into shared
-// memory at `dst` (begin 16-byte aligned), 16 bytes per lane per step.  The
-// last partial 16 bytes, if the array ends there, are copied in 4-byte pieces
-// (elem = 4) or by lane 0 with plain loads and stores (elem = 2).
+// Producer warp: moves each tile with 1-D bulk copies (the copy engine does
+// the work; the issuing lanes spend a few instructions per copy).
+//
+// A stage is filled in `nsub` sub-stages, each with its own full barrier:
+// sub-stage q holds tile rows [2q*PH, 2(q+1)*PH), the rows the consumers'
+// q-th row pair reads, so consumers start on a stage's first rows while the
+// rest is still arriving.  (With nsub = 1 the whole tile, with its leading
+// alignment rows, is one sub-stage.)  Lane q of the producer warp issues
+// sub-stage q, so the lanes' address arithmetic runs side by side.
+//
+// bulk_bytes: the bulk part of copying bytes [begin, end) of an array of
+// `total` bytes (begin 16-byte aligned).  It ends at a 16-byte boundary:
+// rounded up (a few bytes past the tile, never past the array) or, at the
+// very end of the array, rounded down; plain_tail copies what rounding down
+// left with 2-byte loads and stores.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void warp_copy(uint32_t dst, const uint8_t *base,
-                                          long long begin, long long end,
-                                          long long total, int elem, int lane,
-                                          bool &plain) {
+constexpr uint32_t kBulkChunk = 16384;  // bytes per bulk copy instruction
+
+__device__ __forceinline__ uint32_t bulk_bytes(long long begin, long long end,
+                                               long long total) {
   long long e16 = (end + 15) & ~15LL;
   if (e16 > total) e16 = end & ~15LL;
-  for (long long o = begin + 16LL * lane; o < e16; o += 512)
-    cp_async16(dst + static_cast<uint32_t>(o - begin), base + o);
-  for (long long o = (e16 > begin ? e16 : begin) + 4LL * lane; o + 4 <= end;
-       o += 128)
-    if (elem == 4) cp_async4(dst + static_cast<uint32_t>(o - begin), base + o);
-  if (elem == 2 && lane == 0) {
-    for (long long o = e16 > begin ? e16 : begin; o < end; o += 2) {
-      const uint16_t v = *reinterpret_cast<const uint16_t *>(base + o);
-      asm volatile("st.shared.u16 [%0], %1;\n" ::"r"(dst + static_cast<uint32_t>(o - begin)),
-                   "h"(v)
-                   : "memory");
-      plain = true;
-    }
+  return e16 > begin ? static_cast<uint32_t>(e16 - begin) : 0u;
+}
+
+__device__ __noinline__ void plain_tail(uint32_t dst, const uint8_t *src,
+                                        uint32_t from, uint32_t to) {
+  for (uint32_t o = from; o < to; o += 2) {
+    const uint16_t v = *reinterpret_cast<const uint16_t *>(src + o);
+    asm volatile("st.shared.u16 [%0], %1;\n" ::"r"(dst + o), "h"(v) : "memory");
+  }
+  // order the plain stores before later bulk writes to this stage
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const uint8_t *src,
+                                          uint32_t bytes, uint64_t *bar) {
+  for (uint32_t o = 0; o < bytes; o += kBulkChunk) {
+    const uint32_t n = bytes - o < kBulkChunk ? bytes - o : kBulkChunk;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1], %2, [%3];\n" ::"r"(dst + o),
+        "l"(src + o), "r"(n), "r"(smem_u32(bar))
+        : "memory");
   }
 }
 
 template <int MR>
-__device__ void producer_loop(const StreamParams &p, unsigned char *smem,
-                              uint64_t *full, uint64_t *empty, const Groups &g,
-                              int nseg, int lane) {
+__device__ __forceinline__ void producer_loop(const StreamParams &p,
+                                              unsigned char *smem, uint64_t *full,
+                                              uint64_t *empty, const Groups &g,
+                                              int nseg, int lane, int nb2) {
   TileWalker tw;
   tw.init(nseg, p.N, p.RT, p.stages);
   Tile t;
   const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
   const uint32_t base = smem_u32(smem);
+  const uint32_t rb = p.row_bytes, sb = 2u * p.G;
+  const long long wt = p.total_rows * rb, stt = p.total_rows * sb;
+  const int q = lane;  // this lane's sub-stage
+  const bool active = q < p.nsub;
+  const int sub_rows = 2 * p.PH;
+  int issued = 0;
+  bool failed = false;
+  // The first copies wait at named barrier 2 for the consumers' activation
+  // prefetches; the first tile's addresses are worked out before that.
+  bool started = false;
   while (tw.next(t)) {
     const int st = tw.st;
-    if (!mbar_wait(&empty[st], tw.phase ^ 1u)) {
-      if (p.err && lane == 0) atomicOr(p.err, 2);
-      return;
+    // warp-uniform outcome: the lanes leave the loop together
+    if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], tw.phase ^ 1u))) {
+      failed = true;
+      break;
     }
-    const Seg sg = seg_info<MR>(p, g, t.seg);
-    const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
-    const long long ar = abs_row(p, sg.arr, t.row);
-    const int lead = static_cast<int>(ar & (p.RA - 1));  // RA: power of two
-    const long long r0 = ar - lead, r1 = ar + t.nrows;
-    const uint32_t dst = base + st * stage_bytes;
-    const long long sb = 2LL * p.G;
-    bool plain = false;
-    warp_copy(dst, p.w[w_arr], r0 * p.row_bytes, r1 * p.row_bytes,
-              p.total_rows * p.row_bytes, 4, lane, plain);
-    warp_copy(dst + p.w_stage, reinterpret_cast<const uint8_t *>(p.s[w_arr]),
-              r0 * sb, r1 * sb, p.total_rows * sb, 2, lane, plain);
-    warp_copy(dst + p.w_stage + p.s_stage,
-              reinterpret_cast<const uint8_t *>(p.b[w_arr]), r0 * sb, r1 * sb,
-              p.total_rows * sb, 2, lane, plain);
-    // every lane's copies arrive asynchronously; lane 0 also arrives once
-    // for its plain stores (if any), keeping the expected count fixed
-    cp_async_arrive(&full[st]);
-    if (lane == 0) mbar_arrive(&full[st]);
+    uint32_t dw = 0, ds = 0, bw = 0, bs = 0;
+    const uint8_t *wsrc = nullptr, *ssrc = nullptr, *bsrc = nullptr;
+    if (active) {
+      const Seg sg = seg_info<MR>(p, g, t.seg);
+      const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
+      const long long ar = abs_row(p, sg.arr, t.row);
+      const int lead = static_cast<int>(ar & (p.RA - 1));  // RA: power of two
+      // tile-relative rows [lo, hi); the first sub-stage starts at the lead
+      const int lo = q == 0 ? -lead : q * sub_rows;
+      int hi = q == p.nsub - 1 ? t.nrows : (q + 1) * sub_rows;
+      if (hi > t.nrows) hi = t.nrows;
+      if (hi < lo) hi = lo;
+      const long long a0 = ar + lo, a1 = ar + hi;
+      dw = base + st * stage_bytes + static_cast<uint32_t>(lead + lo) * rb;
+      ds = base + st * stage_bytes + p.w_stage + static_cast<uint32_t>(lead + lo) * sb;
+      wsrc = p.w[w_arr] + a0 * rb;
+      ssrc = reinterpret_cast<const uint8_t *>(p.s[w_arr]) + a0 * sb;
+      bsrc = reinterpret_cast<const uint8_t *>(p.b[w_arr]) + a0 * sb;
+      const uint32_t nw = static_cast<uint32_t>((a1 - a0) * rb);
+      const uint32_t ns = static_cast<uint32_t>((a1 - a0) * sb);
+      bw = bulk_bytes(a0 * rb, a1 * rb, wt);
+      bs = bulk_bytes(a0 * sb, a1 * sb, stt);
+      if (bw < nw) plain_tail(dw, wsrc, bw, nw);
+      if (bs < ns) {
+        plain_tail(ds, ssrc, bs, ns);
+        plain_tail(ds + p.s_stage, bsrc, bs, ns);
+      }
+    }
+    if (!started) {
+      named_sync(2, nb2);
+      started = true;
+    }
+    if (active) {
+      uint64_t *bar = &full[st * p.nsub + q];
+      mbar_arrive_expect_tx(bar, bw + 2 * bs);
+      bulk_copy(dw, wsrc, bw, bar);
+      bulk_copy(ds, ssrc, bs, bar);
+      bulk_copy(ds + p.s_stage, bsrc, bs, bar);
+    }
+    ++issued;
     tw.advance_stage();
   }
+  if (!started) named_sync(2, nb2);
+  if (failed && p.err && lane == 0) atomicOr(p.err, 2);
+  // Before the CTA may exit, every copy this lane started must have landed
+  // (consumers normally saw them already).  Use i of stage s is tile number
+  // i * stages + s; its completion is phase parity i & 1.
+  if (active)
+    for (int s = 0; s < p.stages && s < issued; ++s) {
+      const int last = (issued - 1 - s) / p.stages;
+      mbar_wait(&full[s * p.nsub + q], static_cast<uint32_t>(last) & 1u);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -413,18 +462,19 @@ __device__ void producer_loop(const StreamParams &p, unsigned char *smem,
 // partial-sum slot.
 // ---------------------------------------------------------------------------
 template <int MR>
-__device__ void epilogue_loop(const StreamParams &p, unsigned char *smem,
-                              uint64_t *redfull, uint64_t *redempty,
-                              const Groups &g, int nseg, int lane) {
+__device__ __forceinline__ void epilogue_loop(const StreamParams &p,
+                                              unsigned char *smem,
+                                              uint64_t *redfull,
+                                              uint64_t *redempty,
+                                              const Groups &g, int nseg,
+                                              int lane) {
   TileWalker tw;
   tw.init(nseg, p.N, p.RT, p.nred);
   Tile t;
+  bool dead = false;  // as in the consumers: a wait ran out
   while (tw.next(t)) {
     const int st = tw.st;
-    if (!mbar_wait(&redfull[st], tw.phase)) {
-      if (p.err && lane == 0) atomicOr(p.err, 2);
-      return;
-    }
+    if (!dead && !mbar_wait(&redfull[st], tw.phase)) dead = true;
     const Seg sg = seg_info<MR>(p, g, t.seg);
     const float *rb =
         reinterpret_cast<const float *>(smem + p.red_off + st * p.red_stage);
@@ -448,6 +498,7 @@ __device__ void epilogue_loop(const StreamParams &p, unsigned char *smem,
     if (lane == 0) mbar_arrive(&redempty[st]);
     tw.advance_stage();
   }
+  if (dead && p.err) atomicOr(p.err, 2);
 }
 
 // ---------------------------------------------------------------------------
@@ -477,34 +528,72 @@ __device__ __forceinline__ void transpose_reduce(float (&vals)[NV], int lane) {
   }
 }
 
-// The 32 activations of one unit for one activation row (fp32; silu(gate)*up
-// in MODE_SILU).  row < 0 marks an absent row (zeros).
-__device__ __forceinline__ void unit_activations(const StreamParams &p, int u,
-                                                 int row, float (&v)[32]) {
-  if (row < 0 || u >= p.U) {
+// The raw bf16 words of one unit's activations for one activation row (and,
+// in MODE_SILU, of `up`).
+struct UnitRaw {
+  uint4 x[4], up[4];
+  bool valid;
+};
+
+template <bool SILU>
+__device__ __forceinline__ void fetch_unit(const StreamParams &p, int u, int row,
+                                           UnitRaw &r) {
+  r.valid = row >= 0 && u < p.U;
+  if (!r.valid) return;
+  const size_t off = static_cast<size_t>(row) * p.K + static_cast<size_t>(u) * 32;
+  const uint4 *src = reinterpret_cast<const uint4 *>(p.x + off);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) r.x[q] = __ldg(src + q);
+  if constexpr (SILU) {
+    const uint4 *usrc = reinterpret_cast<const uint4 *>(p.up + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r.up[q] = __ldg(usrc + q);
+  }
+}
+
+template <bool SILU>
+__device__ __forceinline__ void prefetch_unit(const StreamParams &p, int u,
+                                              int row) {
+  if (row < 0 || u >= p.U) return;
+  const size_t off = static_cast<size_t>(row) * p.K + static_cast<size_t>(u) * 32;
+  asm volatile("prefetch.global.L1 [%0];\n" ::"l"(p.x + off));
+  if constexpr (SILU)
+    asm volatile("prefetch.global.L1 [%0];\n" ::"l"(p.up + off));
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4 &w, float *v) {
+  const uint32_t xw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    v[2 * h] = __uint_as_float(xw[h] << 16);
+    v[2 * h + 1] = __uint_as_float(xw[h] & 0xffff0000u);
+  }
+}
+
+// The 32 activations of a fetched unit in fp32: x, or v = silu(gate) * up in
+// MODE_SILU (kept in fp32); zeros for an absent row.
+template <bool SILU>
+__device__ __forceinline__ void unit_values(const UnitRaw &r, float (&v)[32]) {
+  if (!r.valid) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = 0.f;
     return;
   }
-  const size_t off = static_cast<size_t>(row) * p.K + static_cast<size_t>(u) * 32;
-  const uint4 *src = reinterpret_cast<const uint4 *>(p.x + off);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 xv = __ldg(src + q);
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  for (int q = 0; q < 4; ++q) unpack_bf16x8(r.x[q], v + 8 * q);
+  if constexpr (SILU) {
+    // silu(g) = g / (1 + e^-g) with the fast exponential and division
+    // intrinsics (relative error near 2^-21, far inside the tolerance); for
+    // g below about -88 the divisor overflows and the result is -0.
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      v[8 * q + 2 * h] = __uint_as_float(xw[h] << 16);
-      v[8 * q + 2 * h + 1] = __uint_as_float(xw[h] & 0xffff0000u);
-    }
-  }
-  if (p.mode == MODE_SILU) {
-    // v = silu(gate) * up, kept in fp32
-    const uint16_t *up = p.up + off;
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-      const float g = v[i];
-      v[i] = g / (1.0f + expf(-g)) * bf16_to_f32(up[i]);
+    for (int q = 0; q < 4; ++q) {
+      float up[8];
+      unpack_bf16x8(r.up[q], up);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float g = v[8 * q + i];
+        v[8 * q + i] = __fdividef(g, 1.0f + __expf(-g)) * up[i];
+      }
     }
   }
 }
@@ -514,7 +603,7 @@ __device__ __forceinline__ void unit_activations(const StreamParams &p, int u,
 // Float path (3/5/6-bit codes): pre-scaled fp32 activations.
 // Both: `back` scales a unit partial back to activation units and
 // vs = (sum of the unit's activations) / back, for the bias term.
-template <int BITS, int MR>
+template <int BITS, int MR, bool SILU>
 struct UnitActs {
   static constexpr bool kInt = kIntPath<BITS>;
   uint32_t dig[kInt ? MR : 1][3][8];
@@ -525,8 +614,10 @@ struct UnitActs {
                                        const int (&rows)[MR]) {
 #pragma unroll
     for (int m = 0; m < MR; ++m) {
+      UnitRaw raw;
+      fetch_unit<SILU>(p, u, rows[m], raw);
       float v[32];
-      unit_activations(p, u, rows[m], v);
+      unit_values<SILU>(raw, v);
       if constexpr (kInt) {
         digits_unit<BITS>(v, dig[m], back[m], vs[m]);
       } else {
@@ -549,12 +640,12 @@ __host__ __device__ constexpr int rows_per_thread() {
 // Partial sums of two rows of the thread's unit: decode, dot products, group
 // scale and bias.  Partials stay in the unit's scale; the caller multiplies
 // by `back` once per tile.
-template <int BITS, int MR>
+template <int BITS, int MR, bool SILU>
 __device__ __forceinline__ void row_pair_dot(const uint32_t (&w0)[BITS],
                                              uint32_t sb0,
                                              const uint32_t (&w1)[BITS],
                                              uint32_t sb1,
-                                             const UnitActs<BITS, MR> &ua,
+                                             const UnitActs<BITS, MR, SILU> &ua,
                                              float *p0, float *p1) {
   float r0[MR], r1[MR];
   if constexpr (kIntPath<BITS>) {
@@ -585,8 +676,9 @@ __device__ __forceinline__ void row_pair_dot(const uint32_t (&w0)[BITS],
 }
 
 // BITS: code width; MR: activation rows per segment (1 or 2); NSL: units per
-// consumer thread (1 or 2).
-template <int BITS, int MR, int NSL>
+// consumer thread (1 or 2); SILU: the activations are silu(gate) * up
+// (MODE_SILU only, a separate kernel so the others carry none of its code).
+template <int BITS, int MR, int NSL, bool SILU>
 __global__ void __launch_bounds__(512, 1)
     qmv_stream_kernel(const StreamParams p) {
   constexpr int RPT = rows_per_thread<BITS, MR, NSL>();
@@ -595,22 +687,11 @@ __global__ void __launch_bounds__(512, 1)
   const int Tc = p.Upad * p.PH / NSL;  // consumer threads
   const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
   uint64_t *full = reinterpret_cast<uint64_t *>(
-      smem + static_cast<size_t>(p.stages) * stage_bytes);
-  uint64_t *empty = full + p.stages;
+      smem + static_cast<size_t>(p.stages) * stage_bytes);  // [stages][nsub]
+  uint64_t *empty = full + p.stages * p.nsub;
   uint64_t *redfull = empty + p.stages;
   uint64_t *redempty = redfull + p.nred;
 
-  if (tid == 0) {
-    for (int i = 0; i < p.stages; ++i) {
-      mbar_init(&full[i], 33);      // 32 async arrivals + lane 0
-      mbar_init(&empty[i], Tc / 32);  // consumer warps
-    }
-    for (int i = 0; i < p.nred; ++i) {
-      mbar_init(&redfull[i], Tc / 32);
-      mbar_init(&redempty[i], 1);   // epilogue warp
-    }
-    fence_mbar_init();
-  }
   Groups g{};
   int nseg;
   if (p.mode == MODE_GATHER) {
@@ -618,16 +699,31 @@ __global__ void __launch_bounds__(512, 1)
     build_groups<MR>(p, g, tid, blockDim.x);  // ends with __syncthreads
     nseg = *g.nseg;
   } else {
-    __syncthreads();
     nseg = p.nmat * p.nch;
   }
 
+  if (tid >= Tc && tid < Tc + 32) {
+    // producer warp: one thread sets up the barriers and starts streaming at
+    // once; the others may use the barriers after named barrier 1
+    if (tid == Tc) {
+      for (int i = 0; i < p.stages * p.nsub; ++i)
+        mbar_init(&full[i], 1);         // the producer's expect-tx arrival
+      for (int i = 0; i < p.stages; ++i)
+        mbar_init(&empty[i], Tc / 32);  // consumer warps
+      for (int i = 0; i < p.nred; ++i) {
+        mbar_init(&redfull[i], Tc / 32);
+        mbar_init(&redempty[i], 1);     // epilogue warp
+      }
+      fence_mbar_init();
+    }
+    __syncwarp();
+    named_arrive(1, blockDim.x);
+    producer_loop<MR>(p, smem, full, empty, g, nseg, tid & 31, Tc + 32);
+    return;
+  }
   if (tid >= Tc) {
-    const int lane = tid & 31;
-    if (tid < Tc + 32)
-      producer_loop<MR>(p, smem, full, empty, g, nseg, lane);
-    else
-      epilogue_loop<MR>(p, smem, redfull, redempty, g, nseg, lane);
+    named_sync(1, blockDim.x);
+    epilogue_loop<MR>(p, smem, redfull, redempty, g, nseg, tid & 31);
     return;
   }
 
@@ -648,12 +744,40 @@ __global__ void __launch_bounds__(512, 1)
   };
   const int nfull = rows_of(p.RT);
 
-  UnitActs<BITS, MR> ua[NSL];
+  UnitActs<BITS, MR, SILU> ua[NSL];
   int loaded = -1;  // key of the activation rows held in ua
 
   TileWalker tw, twr;  // stage ring and partial-sum ring positions
   tw.init(nseg, p.N, p.RT, p.stages);
   twr.init(nseg, p.N, p.RT, p.nred);
+
+  // The first segment's activations are prefetched before the producer
+  // starts the weight stream (named barrier 2), so that these few lines are
+  // not queued behind it in HBM.  The mbarriers are used only after named
+  // barrier 1, which the producer passes once it has set them up.
+  {
+    TileWalker w0 = tw;
+    Tile t0;
+    if (w0.next(t0)) {
+      const Seg sg0 = seg_info<MR>(p, g, t0.seg);
+#pragma unroll
+      for (int j = 0; j < NSL; ++j)
+#pragma unroll
+        for (int m = 0; m < MR; ++m)
+          prefetch_unit<SILU>(p, su[j], seg_xrow<MR>(p, g, sg0, m));
+    }
+    named_arrive(2, Tc + 32);
+  }
+  named_sync(1, blockDim.x);
+
+  // A wait that runs out marks the thread dead: it records the error and
+  // runs to the end without waiting again (results are then garbage), so the
+  // warp stays converged for its shuffles.
+  bool dead = false;
+  auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
+    if (!dead && !mbar_wait(bar, parity)) dead = true;
+  };
+
   Tile t, tr;
   while (tw.next(t)) {
     twr.next(tr);
@@ -671,10 +795,11 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lead = static_cast<uint32_t>(ar & (p.RA - 1));
     const int nvalid = t.nrows == p.RT ? nfull : rows_of(t.nrows);
 
-    if (!mbar_wait(&full[st], tw.phase)) {
-      if (p.err && lane == 0) atomicOr(p.err, 2);
-      return;
-    }
+    uint64_t *fbar = &full[st * p.nsub];
+    // Every warp waits for the stage's first sub-stage, rows or not: its
+    // release of the stage below must not count towards the stage's previous
+    // use, which only the refill (after all warps released it) rules out.
+    wait_bar(fbar, tw.phase);
     const uint32_t wst = smem_base + st * stage_bytes + (lead + ph) * row_bytes;
     const uint32_t sst =
         smem_base + st * stage_bytes + p.w_stage + (lead + ph) * srow_bytes;
@@ -685,26 +810,28 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
     for (int j = 0; j < NSL; ++j) {
       const int u = su[j];
-      if (u < p.U) {
+      if (u < p.U && nvalid > 0) {  // warp-uniform
         float pj[RPT * MR];
 #pragma unroll
         for (int i = 0; i < RPT * MR; ++i) pj[i] = 0.f;
         const uint32_t aw = wst + static_cast<uint32_t>(u) * (4 * BITS);
         const uint32_t as = sst + 2u * static_cast<uint32_t>(u >> p.gs_shift);
+        // Row pairs in order, each after its sub-stage has landed; a pair
+        // past the thread's last row is skipped (warp-uniform), and a lone
+        // last row is computed twice with the copy dropped at the store.
 #pragma unroll
         for (int q = 0; q < RPT / 2; ++q) {
-          if (2 * q < nvalid) {  // warp-uniform
-            // a row past the tile end reuses the pair's first row
-            const int rb = 2 * q + 1 < nvalid ? 2 * q + 1 : 2 * q;
-            uint32_t w0[BITS], w1[BITS];
-            lds_unit<BITS>(aw + 2 * q * rstep, w0);
-            lds_unit<BITS>(aw + rb * rstep, w1);
-            const uint32_t sa = as + 2 * q * sstep, sb = as + rb * sstep;
-            const uint32_t sb0 = lds16(sa) | (lds16(sa + p.s_stage) << 16);
-            const uint32_t sb1 = lds16(sb) | (lds16(sb + p.s_stage) << 16);
-            row_pair_dot<BITS, MR>(w0, sb0, w1, sb1, ua[j], pj + (2 * q) * MR,
-                                   pj + (2 * q + 1) * MR);
-          }
+          if (2 * q >= nvalid) break;
+          const int ra = 2 * q, rb = min(2 * q + 1, nvalid - 1);
+          if (q > 0 && p.nsub > 1) wait_bar(fbar + q, tw.phase);
+          uint32_t w0[BITS], w1[BITS];
+          lds_unit<BITS>(aw + ra * rstep, w0);
+          lds_unit<BITS>(aw + rb * rstep, w1);
+          const uint32_t sa = as + ra * sstep, sb = as + rb * sstep;
+          const uint32_t sb0 = lds16(sa) | (lds16(sa + p.s_stage) << 16);
+          const uint32_t sb1 = lds16(sb) | (lds16(sb + p.s_stage) << 16);
+          row_pair_dot<BITS, MR, SILU>(w0, sb0, w1, sb1, ua[j], pj + (2 * q) * MR,
+                                 pj + (2 * q + 1) * MR);
         }
 #pragma unroll
         for (int i = 0; i < RPT * MR; ++i)
@@ -719,10 +846,7 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int NV = RPT * MR;
     transpose_reduce<NV>(part, lane);
     const int rs = twr.st;
-    if (!mbar_wait(&redempty[rs], twr.phase ^ 1u)) {
-      if (p.err && lane == 0) atomicOr(p.err, 2);
-      return;
-    }
+    wait_bar(&redempty[rs], twr.phase ^ 1u);
     float *rbuf = reinterpret_cast<float *>(smem + p.red_off + rs * p.red_stage);
     if ((lane % (32 / NV)) == 0) {
       const int idx = lane / (32 / NV);
@@ -735,6 +859,7 @@ __global__ void __launch_bounds__(512, 1)
     tw.advance_stage();
     twr.advance_stage();
   }
+  if (dead && p.err) atomicOr(p.err, 2);
 }
 
 }  // namespace qmvk

@@ -172,3 +172,22 @@ def test_gather_empty_is_a_no_op():
                    dev_u32(np.zeros(1, np.uint32)), empty_bf16(1, N), 0, 1, E, N,
                    K, bits, gs)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("bits", [4, 3])
+def test_gather_many_tiny_segments(bits):
+    # 2-row experts and thousands of pairs: every CTA walks more tiny tiles
+    # than its stage ring holds, and most consumer warps have no row in a
+    # tile, so stages are reused while those warps only release them
+    E, N, K, gs, T = 16, 2, 128, 64, 512
+    w, s, b = _moe_inputs(E, N, K, bits, gs, seed=600 + bits)
+    x = synth.normal_bf16((T, K), seed=601)
+    rng = np.random.default_rng(602)
+    P = 4096
+    lhs = rng.integers(0, T, size=P).astype(np.uint32)
+    rhs = rng.integers(0, E, size=P).astype(np.uint32)
+    y, st = _gather(x, w, s, b, lhs, rhs, P, T, E, N, K, bits, gs, False)
+    assert st == 0
+    y_ref, a_ref, valid = oracle.gather(x, w, s, b, lhs, rhs, P, T, E, N, K, bits, gs)
+    assert valid.all()
+    check(y, y_ref, a_ref, f"gather tiny segments bits={bits}")

@@ -92,3 +92,14 @@ def test_qmv_repeatable():
     y1 = run_qmv(x, w, s, b, M, N, K, bits, gs)
     y2 = run_qmv(x, w, s, b, M, N, K, bits, gs)
     assert np.array_equal(y1, y2)
+
+
+def test_qmv_many_chunks_tiny_rows():
+    # M = 8192 activation rows in 4096 chunks of two over N = 2 rows: each CTA
+    # walks more 2-row tiles than its stage ring holds, with most consumer
+    # warps idle in every tile
+    M, N, K, bits, gs = 8192, 2, 128, 4, 32
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=4242)
+    y = run_qmv(x, w, s, b, M, N, K, bits, gs)
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, nthreads=8)
+    check(y, y_ref, a_ref, "qmv many chunks")
