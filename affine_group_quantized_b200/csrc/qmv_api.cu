@@ -113,8 +113,8 @@ struct Plan {
 // Rows per consumer thread per tile; the same rule as the kernel's
 // rows_per_thread<BITS, MR, NSL>().
 int rows_per_thread_host(int bits, int mr, int nsl) {
-  const int base = bits == 2 ? 16 : (bits == 3 || bits == 4) ? 8 : 4;
-  return (mr * nsl == 1) ? base : (base / 2 < 2 ? 2 : base / 2);
+  const int base = (bits == 2 || bits == 3 || bits == 4) ? 16 : 8;
+  return (mr * nsl == 1) ? base : base / 2;
 }
 
 // Thread layout: Upad (>= 32, a multiple of 32) consumer threads cover the
@@ -144,37 +144,37 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   const int RA = ra_w * ra_s / gcd_i(ra_w, ra_s);
   const int wpr = Upad / 32 / nsl;
   // consumer threads: up to 448 (plus producer and epilogue warps: 512 per
-  // CTA, 128 registers per thread), as many row phases as keep the stage
-  // ring at least three tiles deep
+  // CTA, 128 registers per thread).  A slot holds SR rows of every row
+  // phase (SR = 2 * pairs per slot, the kernel's pairs_per_slot<BITS>); the
+  // ring must hold the slots of two tiles (RPT / SR each), so the row phases
+  // are reduced until it does.
+  const int SR = 2 * 2;  // the kernel's 2 * pairs_per_slot<BITS>()
   const int tc_max = 448;
   int PH = nsl == 1 && Upad <= tc_max ? tc_max / Upad : 1;
-  struct Sizes { long long w, s, red, stage; };
+  struct Sizes { long long w, s, red, slot; };
   auto sizes = [&](int ph) {
     Sizes z;
-    const long long rows = static_cast<long long>(RPT) * ph + RA - 1;
-    z.w = (rows * row_bytes + 15 + 15) / 16 * 16;
-    z.s = (rows * 2LL * G + 15 + 15) / 16 * 16;
+    const long long rows = static_cast<long long>(SR) * ph + RA - 1;
+    z.w = (rows * row_bytes + 16 + 15) / 16 * 16;
+    z.s = (rows * 2LL * G + 16 + 15) / 16 * 16;
     z.red = (static_cast<long long>(RPT) * ph * mr * wpr * 4 + 15) / 16 * 16;
-    z.stage = z.w + 2 * z.s;
+    z.slot = z.w + 2 * z.s;
     return z;
   };
   const int nred = 4;
-  // sub-stages (one per row pair of the consumer threads) need every row
-  // start 16-byte aligned
-  const int nsub = (RA == 1 && RPT >= 4) ? RPT / 2 : 1;
-  auto depth_of = [&](int ph) {
+  auto slots_of = [&](int ph) {
     const Sizes z = sizes(ph);
-    return (dev->smem_optin - grp_bytes - 256 - nred * (z.red + 16)) /
-           (z.stage + 8 * (nsub + 1));
+    return (dev->smem_optin - grp_bytes - 256 - nred * (z.red + 16)) / (z.slot + 16);
   };
-  while (PH > 1 && depth_of(PH) < 4) --PH;
+  const int tile_slots_max = (RPT + SR - 1) / SR;
+  while (PH > 1 && slots_of(PH) < 2 * tile_slots_max) --PH;
   const int Tc = Upad * PH / nsl;
   if (Tc > tc_max || Tc % 32 != 0)
     return fail(QMV_ERR_UNSUPPORTED, "K=%d has no thread layout", K);
   const Sizes z = sizes(PH);
-  long long ns = depth_of(PH);
-  if (ns > 12) ns = 12;
-  if (ns < 2)
+  long long ns = slots_of(PH);
+  if (ns > 32) ns = 32;
+  if (ns < tile_slots_max)
     return fail(QMV_ERR_UNSUPPORTED, "shape needs more shared memory than the device offers");
   const int RT = RPT * PH;
   p.gs_shift = 0;
@@ -185,16 +185,15 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   p.PH = PH;
   p.RT = RT;
   p.RA = RA;
-  p.stages = static_cast<int>(ns);
-  p.nsub = nsub;
+  p.nslot = static_cast<int>(ns);
+  p.slot_rows = SR * PH;
   p.wpr = wpr;
   p.row_bytes = static_cast<uint32_t>(row_bytes);
   p.nch = p.mode == qmvk::MODE_GATHER ? 1 : (p.M + mr - 1) / mr;
-  p.w_stage = static_cast<uint32_t>(z.w);
-  p.s_stage = static_cast<uint32_t>(z.s);
-  const long long ring = ns * z.stage;
-  p.red_off = static_cast<uint32_t>(
-      (ring + ((nsub + 1) * ns + 2 * nred) * 8 + 15) / 16 * 16);
+  p.w_slot = static_cast<uint32_t>(z.w);
+  p.s_slot = static_cast<uint32_t>(z.s);
+  const long long ring = ns * z.slot;
+  p.red_off = static_cast<uint32_t>((ring + (2 * ns + 2 * nred) * 8 + 15) / 16 * 16);
   p.red_stage = static_cast<uint32_t>(z.red);
   p.nred = nred;
   p.grp_off = static_cast<uint32_t>(p.red_off + nred * z.red);
@@ -220,6 +219,9 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
     p.RT = static_cast<int>(rte);
   }
   pl.grid = static_cast<int>(grid < 1 ? 1 : grid);
+  // walk constants for the final tile height
+  p.tps = (p.N + p.RT - 1) / p.RT;
+  p.full_slots = (p.RT + p.slot_rows - 1) / p.slot_rows;
   return QMV_OK;
 }
 

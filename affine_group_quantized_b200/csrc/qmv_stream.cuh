@@ -1,23 +1,26 @@
 // qmv_stream.cuh -- the persistent weight-streaming GEMV kernel (CUDA cores).
 //
 // One CTA per SM with three warp roles:
-//   * producer warp: one thread streams tiles of packed weight rows, with
-//     their scales and biases, from HBM into a ring of shared-memory stages
-//     with 1-D bulk copies (a tile is three contiguous byte ranges) that
-//     complete on the stage's mbarrier.  It sets up the barriers itself and
-//     starts the first stages before the other warps are released.
+//   * producer warp: streams the weight rows, with their scales and biases,
+//     from HBM into a ring of shared-memory slots with 1-D bulk copies that
+//     complete on the slot's mbarrier.  A slot holds one or two row pairs of
+//     every consumer row phase; the lanes of the warp fill a tile's slots
+//     side by side.
 //   * consumer warps: each thread owns one 32-code "unit" column of the
 //     weight rows (its activations stay in registers) and a row phase.  It
-//     decodes its unit of its rows of the stage, multiplies with the
+//     decodes its unit of its rows of each slot, multiplies with the
 //     activations (8-bit integer dot products for 2/4/8-bit codes, fp32 FMAs
 //     for 3/5/6-bit codes), applies the group scale and bias, and the warp
-//     reduces the row partials with shuffles into the stage's partial-sum
-//     buffer;
+//     reduces the tile's row partials with shuffles into a partial-sum
+//     ring slot;
 //   * epilogue warp: adds the per-warp partials of each output in a fixed
 //     order, adds the residual if any, rounds once to bf16 and stores.
-// Stage handoffs are mbarrier phases; consumer warps never wait for each
-// other.  Tiles are dealt to CTAs round-robin, so that at any moment all SMs
-// stream from one compact window of memory.
+// Slot and partial-sum handoffs are mbarrier phases; consumer warps never
+// wait for each other.  Copies move in slots (small, so consumers start soon
+// after the first bytes land) while the shuffle reduction and the hand-off
+// to the epilogue happen once per tile (many slots).  Tiles are dealt to
+// CTAs round-robin, so that at any moment all SMs stream from one compact
+// window of memory.
 //
 // The same kernel serves every entry point through `mode`:
 //   MODE_QMV      y = x @ dequant(W).T
@@ -57,16 +60,18 @@ struct StreamParams {
   int U, Upad;            // units per row (K/32) and padded count (>= 32)
   int PH;                 // row phases: Upad threads per row, PH rows at once
   int RT;                 // rows per tile (at most RPT * PH)
+  int tps;                // tiles per segment: ceil(N / RT)
+  int full_slots;         // slots of a full tile: ceil(RT / slot_rows)
   int RA;                 // row alignment making copy starts 16-byte aligned
   int nmat;               // weight matrices (1, or 2 for gate/up)
   int nch;                // activation chunks per matrix: ceil(M / MR)
-  int stages;             // depth of the stage ring
-  int nsub;               // sub-stages per stage (1, or rows-per-thread / 2)
+  int nslot;              // slots in the shared-memory weight ring
+  int slot_rows;          // rows per slot: SR rows of every phase (SR * PH)
   int wpr;                // partial-sum slots per row (consumer warps per row)
   uint32_t row_bytes;     // K * bits / 8
   long long total_rows;   // rows in each weight array (N, or E*N)
   int num_pairs, num_x_rows, num_experts;
-  uint32_t w_stage, s_stage;  // bytes of the W and of the S (= B) region
+  uint32_t w_slot, s_slot;    // bytes of a slot's W and S (= B) regions
   uint32_t red_off;           // smem offset of the partial-sum ring
   uint32_t red_stage;         // bytes of one partial-sum ring slot
   int nred;                   // slots in the partial-sum ring
@@ -90,14 +95,15 @@ struct TileWalker {
   int stages, st;
   uint32_t phase;
 
-  __device__ __forceinline__ void init(int nseg_, int N_, int RT_, int stages_) {
+  __device__ __forceinline__ void init(int nseg_, int N_, int RT_, int tps_,
+                                       int stages_) {
     N = N_;
     RT = RT_;
     nseg = nseg_;
     stages = stages_;
-    tps = (N + RT - 1) / RT;
+    tps = tps_;
     step = gridDim.x;
-    seg = blockIdx.x / tps;
+    seg = static_cast<int>(blockIdx.x) < tps ? 0 : static_cast<int>(blockIdx.x) / tps;
     tj = blockIdx.x - seg * tps;
     st = 0;
     phase = 0;
@@ -108,9 +114,10 @@ struct TileWalker {
     t.row = tj * RT;
     t.nrows = N - t.row < RT ? N - t.row : RT;
     tj += step;
-    while (tj >= tps) {
-      tj -= tps;
-      ++seg;
+    if (tj >= tps) {
+      const int d = tj / tps;
+      tj -= d * tps;
+      seg += d;
     }
     return true;
   }
@@ -121,6 +128,26 @@ struct TileWalker {
     }
   }
 };
+
+// Position in the slot ring: slot k of the walk is slot k % nslot, in its
+// use k / nslot, whose completion is phase parity (k / nslot) & 1.
+struct SlotPos {
+  int idx;
+  uint32_t phase;
+  __device__ __forceinline__ SlotPos plus(int n, int nslot) const {
+    SlotPos r{idx + n, phase};
+    while (r.idx >= nslot) {
+      r.idx -= nslot;
+      r.phase ^= 1u;
+    }
+    return r;
+  }
+};
+
+// Slots of a tile of n rows (a full tile's count is precomputed).
+__device__ __forceinline__ int tile_slots(const StreamParams &p, int n) {
+  return n == p.RT ? p.full_slots : (n + p.slot_rows - 1) / p.slot_rows;
+}
 
 // ---------------------------------------------------------------------------
 // Gather grouping (MODE_GATHER), computed redundantly by every CTA from the
@@ -328,21 +355,20 @@ __device__ __forceinline__ void lds_unit(uint32_t a, uint32_t (&wd)[BITS]) {
 }
 
 // ---------------------------------------------------------------------------
-// Producer warp: moves each tile with 1-D bulk copies (the copy engine does
-// the work; the issuing lanes spend a few instructions per copy).
+// Producer warp: moves the weight rows with 1-D bulk copies (the copy engine
+// does the work; the issuing lanes spend a few instructions per copy).
 //
-// A stage is filled in `nsub` sub-stages, each with its own full barrier:
-// sub-stage q holds tile rows [2q*PH, 2(q+1)*PH), the rows the consumers'
-// q-th row pair reads, so consumers start on a stage's first rows while the
-// rest is still arriving.  (With nsub = 1 the whole tile, with its leading
-// alignment rows, is one sub-stage.)  Lane q of the producer warp issues
-// sub-stage q, so the lanes' address arithmetic runs side by side.
+// Slot q of a tile holds tile rows [q*slot_rows, (q+1)*slot_rows) (fewer at
+// the tile's end), i.e. SR consecutive rows of every consumer row phase, with
+// their scales and biases.  A slot's copy starts at the 16-byte-aligned row
+// at or before its first row (`lead` rows earlier).  Lane q fills slot q of
+// the tile, so the lanes' waits and address arithmetic run side by side.
 //
 // bulk_bytes: the bulk part of copying bytes [begin, end) of an array of
 // `total` bytes (begin 16-byte aligned).  It ends at a 16-byte boundary:
-// rounded up (a few bytes past the tile, never past the array) or, at the
-// very end of the array, rounded down; plain_tail copies what rounding down
-// left with 2-byte loads and stores.
+// rounded up (a few bytes past the slot's rows, never past the array) or,
+// at the very end of the array, rounded down; plain_tail copies what
+// rounding down left with 2-byte loads and stores.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kBulkChunk = 16384;  // bytes per bulk copy instruction
 
@@ -359,7 +385,7 @@ __device__ __noinline__ void plain_tail(uint32_t dst, const uint8_t *src,
     const uint16_t v = *reinterpret_cast<const uint16_t *>(src + o);
     asm volatile("st.shared.u16 [%0], %1;\n" ::"r"(dst + o), "h"(v) : "memory");
   }
-  // order the plain stores before later bulk writes to this stage
+  // order the plain stores before later bulk writes to this slot
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
@@ -379,26 +405,27 @@ template <int MR>
 __device__ __forceinline__ void producer_loop(const StreamParams &p,
                                               unsigned char *smem, uint64_t *full,
                                               uint64_t *empty, const Groups &g,
-                                              int nseg, int lane, int nb2) {
+                                              int nseg, int lane) {
   TileWalker tw;
-  tw.init(nseg, p.N, p.RT, p.stages);
+  tw.init(nseg, p.N, p.RT, p.tps, 1);
   Tile t;
-  const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
+  const uint32_t slot_bytes = p.w_slot + 2 * p.s_slot;
   const uint32_t base = smem_u32(smem);
   const uint32_t rb = p.row_bytes, sb = 2u * p.G;
   const long long wt = p.total_rows * rb, stt = p.total_rows * sb;
-  const int q = lane;  // this lane's sub-stage
-  const bool active = q < p.nsub;
-  const int sub_rows = 2 * p.PH;
-  int issued = 0;
+  const int q = lane;  // this lane's slot within a tile
+  SlotPos pos{0, 0u};
+  long long nslots = 0;  // slots filled so far
   bool failed = false;
-  // The first copies wait at named barrier 2 for the consumers' activation
-  // prefetches; the first tile's addresses are worked out before that.
-  bool started = false;
   while (tw.next(t)) {
-    const int st = tw.st;
+    const int ns_t = tile_slots(p, t.nrows);
+    const bool active = q < ns_t;
+    const SlotPos my = pos.plus(q, p.nslot);
+    bool ok = true;
+    // a slot's first use needs no wait
+    if (active && nslots + q >= p.nslot) ok = mbar_wait(&empty[my.idx], my.phase ^ 1u);
     // warp-uniform outcome: the lanes leave the loop together
-    if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], tw.phase ^ 1u))) {
+    if (!__all_sync(0xffffffffu, ok)) {
       failed = true;
       break;
     }
@@ -407,16 +434,12 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
     if (active) {
       const Seg sg = seg_info<MR>(p, g, t.seg);
       const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
-      const long long ar = abs_row(p, sg.arr, t.row);
-      const int lead = static_cast<int>(ar & (p.RA - 1));  // RA: power of two
-      // tile-relative rows [lo, hi); the first sub-stage starts at the lead
-      const int lo = q == 0 ? -lead : q * sub_rows;
-      int hi = q == p.nsub - 1 ? t.nrows : (q + 1) * sub_rows;
-      if (hi > t.nrows) hi = t.nrows;
-      if (hi < lo) hi = lo;
-      const long long a0 = ar + lo, a1 = ar + hi;
-      dw = base + st * stage_bytes + static_cast<uint32_t>(lead + lo) * rb;
-      ds = base + st * stage_bytes + p.w_stage + static_cast<uint32_t>(lead + lo) * sb;
+      const long long a = abs_row(p, sg.arr, t.row) + q * p.slot_rows;
+      const int lead = static_cast<int>(a & (p.RA - 1));  // RA: power of two
+      const int rows = min(p.slot_rows, t.nrows - q * p.slot_rows);
+      const long long a0 = a - lead, a1 = a + rows;
+      dw = base + my.idx * slot_bytes;
+      ds = dw + p.w_slot;
       wsrc = p.w[w_arr] + a0 * rb;
       ssrc = reinterpret_cast<const uint8_t *>(p.s[w_arr]) + a0 * sb;
       bsrc = reinterpret_cast<const uint8_t *>(p.b[w_arr]) + a0 * sb;
@@ -427,33 +450,27 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
       if (bw < nw) plain_tail(dw, wsrc, bw, nw);
       if (bs < ns) {
         plain_tail(ds, ssrc, bs, ns);
-        plain_tail(ds + p.s_stage, bsrc, bs, ns);
+        plain_tail(ds + p.s_slot, bsrc, bs, ns);
       }
     }
-    if (!started) {
-      named_sync(2, nb2);
-      started = true;
-    }
     if (active) {
-      uint64_t *bar = &full[st * p.nsub + q];
+      uint64_t *bar = &full[my.idx];
       mbar_arrive_expect_tx(bar, bw + 2 * bs);
       bulk_copy(dw, wsrc, bw, bar);
       bulk_copy(ds, ssrc, bs, bar);
-      bulk_copy(ds + p.s_stage, bsrc, bs, bar);
+      bulk_copy(ds + p.s_slot, bsrc, bs, bar);
     }
-    ++issued;
-    tw.advance_stage();
+    pos = pos.plus(ns_t, p.nslot);
+    nslots += ns_t;
   }
-  if (!started) named_sync(2, nb2);
   if (failed && p.err && lane == 0) atomicOr(p.err, 2);
-  // Before the CTA may exit, every copy this lane started must have landed
-  // (consumers normally saw them already).  Use i of stage s is tile number
-  // i * stages + s; its completion is phase parity i & 1.
-  if (active)
-    for (int s = 0; s < p.stages && s < issued; ++s) {
-      const int last = (issued - 1 - s) / p.stages;
-      mbar_wait(&full[s * p.nsub + q], static_cast<uint32_t>(last) & 1u);
-    }
+  // Before the CTA may exit, every copy the warp started must have landed
+  // (consumers normally saw them already): wait for the last use of every
+  // slot that was used.
+  for (int i = lane; i < p.nslot && i < nslots; i += 32) {
+    const long long last = (nslots - 1 - i) / p.nslot;
+    mbar_wait(&full[i], static_cast<uint32_t>(last & 1));
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -469,7 +486,7 @@ __device__ __forceinline__ void epilogue_loop(const StreamParams &p,
                                               const Groups &g, int nseg,
                                               int lane) {
   TileWalker tw;
-  tw.init(nseg, p.N, p.RT, p.nred);
+  tw.init(nseg, p.N, p.RT, p.tps, p.nred);
   Tile t;
   bool dead = false;  // as in the consumers: a wait ran out
   while (tw.next(t)) {
@@ -505,6 +522,16 @@ __device__ __forceinline__ void epilogue_loop(const StreamParams &p,
 // Consumers
 // ---------------------------------------------------------------------------
 
+// c ? a : b on values, kept a register select (a select between two array
+// elements may otherwise become an indexed load from local memory).
+__device__ __forceinline__ float select_f32(bool c, float a, float b) {
+  float r;
+  asm("{\n.reg .pred q;\nsetp.ne.u32 q, %3, 0;\nselp.f32 %0, %1, %2, q;\n}\n"
+      : "=f"(r)
+      : "f"(a), "f"(b), "r"(static_cast<uint32_t>(c)));
+  return r;
+}
+
 // Transposed butterfly over the 32 lanes of a warp: NV partial sums per lane
 // in; afterwards lane l holds the full sum of value l / (32 / NV) in vals[0].
 template <int NV>
@@ -517,8 +544,9 @@ __device__ __forceinline__ void transpose_reduce(float (&vals)[NV], int lane) {
       const bool upper = (lane & off) != 0;
 #pragma unroll
       for (int i = 0; i < n / 2; ++i) {
-        const float send = upper ? vals[i] : vals[i + n / 2];
-        const float keep = upper ? vals[i + n / 2] : vals[i];
+        const float lo = vals[i], hi = vals[i + n / 2];
+        const float send = select_f32(upper, lo, hi);
+        const float keep = select_f32(upper, hi, lo);
         vals[i] = keep + __shfl_xor_sync(full, send, off);
       }
       n >>= 1;
@@ -549,16 +577,6 @@ __device__ __forceinline__ void fetch_unit(const StreamParams &p, int u, int row
 #pragma unroll
     for (int q = 0; q < 4; ++q) r.up[q] = __ldg(usrc + q);
   }
-}
-
-template <bool SILU>
-__device__ __forceinline__ void prefetch_unit(const StreamParams &p, int u,
-                                              int row) {
-  if (row < 0 || u >= p.U) return;
-  const size_t off = static_cast<size_t>(row) * p.K + static_cast<size_t>(u) * 32;
-  asm volatile("prefetch.global.L1 [%0];\n" ::"l"(p.x + off));
-  if constexpr (SILU)
-    asm volatile("prefetch.global.L1 [%0];\n" ::"l"(p.up + off));
 }
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4 &w, float *v) {
@@ -630,11 +648,19 @@ struct UnitActs {
   }
 };
 
-// Rows per consumer thread per tile (a compile-time constant per code width).
+// Row pairs per consumer thread in one slot: two, so that the per-slot wait,
+// release, address arithmetic and reduction are shared by four rows.
+template <int BITS>
+__host__ __device__ constexpr int pairs_per_slot() {
+  return 2;
+}
+
+// Rows per consumer thread per tile (a compile-time constant per code width):
+// the rows handed to the epilogue at once.
 template <int BITS, int MR, int NSL>
 __host__ __device__ constexpr int rows_per_thread() {
-  constexpr int base = BITS == 2 ? 16 : (BITS == 3 || BITS == 4) ? 8 : 4;
-  return (MR * NSL == 1) ? base : (base / 2 < 2 ? 2 : base / 2);
+  constexpr int base = (BITS == 2 || BITS == 3 || BITS == 4) ? 16 : 8;
+  return (MR * NSL == 1) ? base : base / 2;
 }
 
 // Partial sums of two rows of the thread's unit: decode, dot products, group
@@ -685,11 +711,11 @@ __global__ void __launch_bounds__(512, 1)
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
   const int Tc = p.Upad * p.PH / NSL;  // consumer threads
-  const uint32_t stage_bytes = p.w_stage + 2 * p.s_stage;
+  const uint32_t slot_bytes = p.w_slot + 2 * p.s_slot;
   uint64_t *full = reinterpret_cast<uint64_t *>(
-      smem + static_cast<size_t>(p.stages) * stage_bytes);  // [stages][nsub]
-  uint64_t *empty = full + p.stages * p.nsub;
-  uint64_t *redfull = empty + p.stages;
+      smem + static_cast<size_t>(p.nslot) * slot_bytes);
+  uint64_t *empty = full + p.nslot;
+  uint64_t *redfull = empty + p.nslot;
   uint64_t *redempty = redfull + p.nred;
 
   Groups g{};
@@ -703,22 +729,22 @@ __global__ void __launch_bounds__(512, 1)
   }
 
   if (tid >= Tc && tid < Tc + 32) {
-    // producer warp: one thread sets up the barriers and starts streaming at
-    // once; the others may use the barriers after named barrier 1
-    if (tid == Tc) {
-      for (int i = 0; i < p.stages * p.nsub; ++i)
-        mbar_init(&full[i], 1);         // the producer's expect-tx arrival
-      for (int i = 0; i < p.stages; ++i)
-        mbar_init(&empty[i], Tc / 32);  // consumer warps
-      for (int i = 0; i < p.nred; ++i) {
-        mbar_init(&redfull[i], Tc / 32);
-        mbar_init(&redempty[i], 1);     // epilogue warp
-      }
-      fence_mbar_init();
+    // producer warp: its lanes set up the barriers side by side, then it
+    // starts streaming at once; the other warps use the barriers only after
+    // named barrier 1
+    const int lane = tid & 31;
+    for (int i = lane; i < p.nslot; i += 32) {
+      mbar_init(&full[i], 1);         // the producer lane's expect-tx arrival
+      mbar_init(&empty[i], Tc / 32);  // consumer warps
     }
+    for (int i = lane; i < p.nred; i += 32) {
+      mbar_init(&redfull[i], Tc / 32);
+      mbar_init(&redempty[i], 1);     // epilogue warp
+    }
+    fence_mbar_init();
     __syncwarp();
     named_arrive(1, blockDim.x);
-    producer_loop<MR>(p, smem, full, empty, g, nseg, tid & 31, Tc + 32);
+    producer_loop<MR>(p, smem, full, empty, g, nseg, tid & 31);
     return;
   }
   if (tid >= Tc) {
@@ -747,26 +773,26 @@ __global__ void __launch_bounds__(512, 1)
   UnitActs<BITS, MR, SILU> ua[NSL];
   int loaded = -1;  // key of the activation rows held in ua
 
-  TileWalker tw, twr;  // stage ring and partial-sum ring positions
-  tw.init(nseg, p.N, p.RT, p.stages);
-  twr.init(nseg, p.N, p.RT, p.nred);
+  TileWalker tw, twr;  // tiles, and the partial-sum ring position
+  tw.init(nseg, p.N, p.RT, p.tps, 1);
+  twr.init(nseg, p.N, p.RT, p.tps, p.nred);
 
-  // The first segment's activations are prefetched before the producer
-  // starts the weight stream (named barrier 2), so that these few lines are
-  // not queued behind it in HBM.  The mbarriers are used only after named
-  // barrier 1, which the producer passes once it has set them up.
+  // The first segment's activations are loaded straight away, while the
+  // producer sets up and starts the weight stream, so that these few lines
+  // are not queued behind it in HBM.  The mbarriers are used only after
+  // named barrier 1, which the producer passes once it has set them up.
   {
     TileWalker w0 = tw;
     Tile t0;
     if (w0.next(t0)) {
       const Seg sg0 = seg_info<MR>(p, g, t0.seg);
+      int xr[MR];
 #pragma unroll
-      for (int j = 0; j < NSL; ++j)
+      for (int m = 0; m < MR; ++m) xr[m] = seg_xrow<MR>(p, g, sg0, m);
 #pragma unroll
-        for (int m = 0; m < MR; ++m)
-          prefetch_unit<SILU>(p, su[j], seg_xrow<MR>(p, g, sg0, m));
+      for (int j = 0; j < NSL; ++j) ua[j].load(p, su[j], xr);
+      loaded = sg0.key;
     }
-    named_arrive(2, Tc + 32);
   }
   named_sync(1, blockDim.x);
 
@@ -778,10 +804,10 @@ __global__ void __launch_bounds__(512, 1)
     if (!dead && !mbar_wait(bar, parity)) dead = true;
   };
 
+  SlotPos pos{0, 0u};
   Tile t, tr;
   while (tw.next(t)) {
     twr.next(tr);
-    const int st = tw.st;
     const Seg sg = seg_info<MR>(p, g, t.seg);
     if (sg.key != loaded) {
       int xr[MR];
@@ -792,71 +818,86 @@ __global__ void __launch_bounds__(512, 1)
       loaded = sg.key;
     }
     const long long ar = abs_row(p, sg.arr, t.row);
-    const uint32_t lead = static_cast<uint32_t>(ar & (p.RA - 1));
     const int nvalid = t.nrows == p.RT ? nfull : rows_of(t.nrows);
+    const int ns_t = tile_slots(p, t.nrows);
 
-    uint64_t *fbar = &full[st * p.nsub];
-    // Every warp waits for the stage's first sub-stage, rows or not: its
-    // release of the stage below must not count towards the stage's previous
-    // use, which only the refill (after all warps released it) rules out.
-    wait_bar(fbar, tw.phase);
-    const uint32_t wst = smem_base + st * stage_bytes + (lead + ph) * row_bytes;
-    const uint32_t sst =
-        smem_base + st * stage_bytes + p.w_stage + (lead + ph) * srow_bytes;
-
-    float part[RPT * MR];
-#pragma unroll
-    for (int i = 0; i < RPT * MR; ++i) part[i] = 0.f;
-#pragma unroll
-    for (int j = 0; j < NSL; ++j) {
-      const int u = su[j];
-      if (u < p.U && nvalid > 0) {  // warp-uniform
-        float pj[RPT * MR];
-#pragma unroll
-        for (int i = 0; i < RPT * MR; ++i) pj[i] = 0.f;
-        const uint32_t aw = wst + static_cast<uint32_t>(u) * (4 * BITS);
-        const uint32_t as = sst + 2u * static_cast<uint32_t>(u >> p.gs_shift);
-        // Row pairs in order, each after its sub-stage has landed; a pair
-        // past the thread's last row is skipped (warp-uniform), and a lone
-        // last row is computed twice with the copy dropped at the store.
-#pragma unroll
-        for (int q = 0; q < RPT / 2; ++q) {
-          if (2 * q >= nvalid) break;
-          const int ra = 2 * q, rb = min(2 * q + 1, nvalid - 1);
-          if (q > 0 && p.nsub > 1) wait_bar(fbar + q, tw.phase);
-          uint32_t w0[BITS], w1[BITS];
-          lds_unit<BITS>(aw + ra * rstep, w0);
-          lds_unit<BITS>(aw + rb * rstep, w1);
-          const uint32_t sa = as + ra * sstep, sb = as + rb * sstep;
-          const uint32_t sb0 = lds16(sa) | (lds16(sa + p.s_stage) << 16);
-          const uint32_t sb1 = lds16(sb) | (lds16(sb + p.s_stage) << 16);
-          row_pair_dot<BITS, MR, SILU>(w0, sb0, w1, sb1, ua[j], pj + (2 * q) * MR,
-                                 pj + (2 * q + 1) * MR);
-        }
-#pragma unroll
-        for (int i = 0; i < RPT * MR; ++i)
-          part[i] = fmaf(pj[i], ua[j].back[i % MR], part[i]);
-      }
-    }
-    // done reading the stage's weights, scales and biases
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-
-    // ---- reduce over the warp's units; one partial per row and x row ----
-    constexpr int NV = RPT * MR;
-    transpose_reduce<NV>(part, lane);
+    // Slot q holds the thread's rows SR*q .. SR*q + SR-1 (SR = 2 * pairs per
+    // slot).  For each slot: wait, compute its rows' partials, release it,
+    // reduce the partials over the warp's units with a small shuffle
+    // butterfly and write them to the tile's partial-sum slot.  The slot
+    // loop stays rolled (a compact body stays in the instruction cache).
+    // Every warp waits for and releases every slot of the tile, rows or not:
+    // a release must not count towards the slot's previous use, which only
+    // the refill (after all warps released it) rules out.  Rows past the
+    // thread's last row re-read its last row and are dropped at the store.
+    constexpr int SPS = pairs_per_slot<BITS>();
+    constexpr int SR = 2 * SPS;     // thread rows per slot
+    constexpr int NV = SR * MR;     // partials per thread per slot
     const int rs = twr.st;
     wait_bar(&redempty[rs], twr.phase ^ 1u);
     float *rbuf = reinterpret_cast<float *>(smem + p.red_off + rs * p.red_stage);
-    if ((lane % (32 / NV)) == 0) {
-      const int idx = lane / (32 / NV);
-      const int rr = idx / MR, m = idx % MR;
-      const int r = ph + rr * p.PH;
-      if (r < t.nrows) rbuf[(r * MR + m) * p.wpr + wslot] = part[0];
+#pragma unroll 1
+    for (int q = 0; q < ns_t; ++q) {
+      const SlotPos my = pos.plus(q, p.nslot);
+      wait_bar(&full[my.idx], my.phase);
+      const int nv = nvalid - SR * q;  // thread rows in this slot (may be <= 0)
+      float part[NV];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) part[i] = 0.f;
+      if (nv > 0) {  // warp-uniform
+        const uint32_t lead =
+            static_cast<uint32_t>((ar + q * p.slot_rows) & (p.RA - 1));
+        const uint32_t sl = smem_base + my.idx * slot_bytes;
+        const uint32_t wrow = sl + (lead + ph) * row_bytes;
+        const uint32_t srow = sl + p.w_slot + (lead + ph) * srow_bytes;
+#pragma unroll
+        for (int j = 0; j < NSL; ++j) {
+          const int u = su[j];
+          if (u < p.U) {
+            const uint32_t aw = wrow + static_cast<uint32_t>(u) * (4 * BITS);
+            const uint32_t as = srow + 2u * static_cast<uint32_t>(u >> p.gs_shift);
+#pragma unroll
+            for (int k = 0; k < SPS; ++k) {
+              if (2 * k < nv) {  // warp-uniform
+                const int ra = 2 * k, rb = 2 * k + 1 < nv ? 2 * k + 1 : 2 * k;
+                uint32_t w0[BITS], w1[BITS];
+                lds_unit<BITS>(aw + ra * rstep, w0);
+                lds_unit<BITS>(aw + rb * rstep, w1);
+                const uint32_t sa = as + ra * sstep, sb = as + rb * sstep;
+                const uint32_t sb0 = lds16(sa) | (lds16(sa + p.s_slot) << 16);
+                const uint32_t sb1 = lds16(sb) | (lds16(sb + p.s_slot) << 16);
+                float d0[MR], d1[MR];
+#pragma unroll
+                for (int m = 0; m < MR; ++m) d0[m] = d1[m] = 0.f;
+                row_pair_dot<BITS, MR, SILU>(w0, sb0, w1, sb1, ua[j], d0, d1);
+                // back to activation units (per unit)
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+                  part[(2 * k) * MR + m] =
+                      fmaf(d0[m], ua[j].back[m], part[(2 * k) * MR + m]);
+                  part[(2 * k + 1) * MR + m] =
+                      fmaf(d1[m], ua[j].back[m], part[(2 * k + 1) * MR + m]);
+                }
+              }
+            }
+          }
+        }
+      }
+      // done reading the slot
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[my.idx]);
+      // ---- one partial per row and x row over the warp's units ----
+      transpose_reduce<NV>(part, lane);
+      if ((lane % (32 / NV)) == 0) {
+        const int idx = lane / (32 / NV);
+        const int rr = idx / MR, m = idx % MR;
+        const int r = ph + (SR * q + rr) * p.PH;
+        if (rr < nv && r < t.nrows) rbuf[(r * MR + m) * p.wpr + wslot] = part[0];
+      }
     }
+    pos = pos.plus(ns_t, p.nslot);
     __syncwarp();
     if (lane == 0) mbar_arrive(&redfull[rs]);
-    tw.advance_stage();
     twr.advance_stage();
   }
   if (dead && p.err) atomicOr(p.err, 2);
