@@ -80,9 +80,12 @@ struct StreamParams {
 
 // ---------------------------------------------------------------------------
 // Tiles.  A segment has tps = ceil(N / RT) tiles; the tiles of all segments
-// are numbered segment by segment and dealt round-robin: CTA c gets tiles
-// c, c + G, c + 2G, ...  Every role of a CTA runs the same walk and uses the
-// tile's position in it as its stage index.
+// are numbered segment by segment.  They are dealt to CTAs round-robin (CTA
+// c gets tiles c, c + G, c + 2G, ...), so that at any moment all SMs stream
+// from one compact window of memory -- or, for the gather mode's many short
+// segments, in contiguous blocks (CTA c gets tiles [c*B, (c+1)*B)), so that
+// a CTA's consecutive tiles mostly share a segment and its activations.
+// Every role of a CTA runs the same walk.
 // ---------------------------------------------------------------------------
 struct Tile {
   int seg;    // segment index
@@ -91,25 +94,38 @@ struct Tile {
 };
 
 struct TileWalker {
-  int seg, tj, tps, nseg, step, N, RT;
+  int seg, tj, tps, nseg, step, N, RT, left;
   int stages, st;
   uint32_t phase;
 
   __device__ __forceinline__ void init(int nseg_, int N_, int RT_, int tps_,
-                                       int stages_) {
+                                       int stages_, bool blocked = false) {
     N = N_;
     RT = RT_;
     nseg = nseg_;
     stages = stages_;
     tps = tps_;
-    step = gridDim.x;
-    seg = static_cast<int>(blockIdx.x) < tps ? 0 : static_cast<int>(blockIdx.x) / tps;
-    tj = blockIdx.x - seg * tps;
     st = 0;
     phase = 0;
+    if (blocked) {
+      const int total = nseg * tps;
+      const int B = (total + gridDim.x - 1) / gridDim.x;
+      const int start = static_cast<int>(blockIdx.x) * B;
+      left = total - start < B ? total - start : B;
+      if (left < 0) left = 0;
+      step = 1;
+      seg = start < total ? start / tps : nseg;
+      tj = start < total ? start - seg * tps : 0;
+    } else {
+      left = 0x7fffffff;
+      step = gridDim.x;
+      seg = static_cast<int>(blockIdx.x) < tps ? 0 : static_cast<int>(blockIdx.x) / tps;
+      tj = blockIdx.x - seg * tps;
+    }
   }
   __device__ __forceinline__ bool next(Tile &t) {
-    if (seg >= nseg) return false;
+    if (seg >= nseg || left <= 0) return false;
+    --left;
     t.seg = seg;
     t.row = tj * RT;
     t.nrows = N - t.row < RT ? N - t.row : RT;
@@ -407,7 +423,7 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
                                               uint64_t *empty, const Groups &g,
                                               int nseg, int lane) {
   TileWalker tw;
-  tw.init(nseg, p.N, p.RT, p.tps, 1);
+  tw.init(nseg, p.N, p.RT, p.tps, 1, p.mode == MODE_GATHER);
   Tile t;
   const uint32_t slot_bytes = p.w_slot + 2 * p.s_slot;
   const uint32_t base = smem_u32(smem);
@@ -486,7 +502,7 @@ __device__ __forceinline__ void epilogue_loop(const StreamParams &p,
                                               const Groups &g, int nseg,
                                               int lane) {
   TileWalker tw;
-  tw.init(nseg, p.N, p.RT, p.tps, p.nred);
+  tw.init(nseg, p.N, p.RT, p.tps, p.nred, p.mode == MODE_GATHER);
   Tile t;
   bool dead = false;  // as in the consumers: a wait ran out
   while (tw.next(t)) {
@@ -774,8 +790,8 @@ __global__ void __launch_bounds__(512, 1)
   int loaded = -1;  // key of the activation rows held in ua
 
   TileWalker tw, twr;  // tiles, and the partial-sum ring position
-  tw.init(nseg, p.N, p.RT, p.tps, 1);
-  twr.init(nseg, p.N, p.RT, p.tps, p.nred);
+  tw.init(nseg, p.N, p.RT, p.tps, 1, p.mode == MODE_GATHER);
+  twr.init(nseg, p.N, p.RT, p.tps, p.nred, p.mode == MODE_GATHER);
 
   // The first segment's activations are loaded straight away, while the
   // producer sets up and starts the weight stream, so that these few lines
