@@ -789,9 +789,11 @@ __global__ void __launch_bounds__(512, 1)
   UnitActs<BITS, MR, SILU> ua[NSL];
   int loaded = -1;  // key of the activation rows held in ua
 
-  TileWalker tw, twr;  // tiles, and the partial-sum ring position
+  TileWalker tw;
   tw.init(nseg, p.N, p.RT, p.tps, 1, p.mode == MODE_GATHER);
-  twr.init(nseg, p.N, p.RT, p.tps, p.nred, p.mode == MODE_GATHER);
+  // partial-sum ring position of the current tile: slot and phase parity
+  int rs = 0;
+  uint32_t rphase = 0;
 
   // The first segment's activations are loaded straight away, while the
   // producer sets up and starts the weight stream, so that these few lines
@@ -821,9 +823,8 @@ __global__ void __launch_bounds__(512, 1)
   };
 
   SlotPos pos{0, 0u};
-  Tile t, tr;
+  Tile t;
   while (tw.next(t)) {
-    twr.next(tr);
     const Seg sg = seg_info<MR>(p, g, t.seg);
     if (sg.key != loaded) {
       int xr[MR];
@@ -849,8 +850,7 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int SPS = pairs_per_slot<BITS>();
     constexpr int SR = 2 * SPS;     // thread rows per slot
     constexpr int NV = SR * MR;     // partials per thread per slot
-    const int rs = twr.st;
-    wait_bar(&redempty[rs], twr.phase ^ 1u);
+    wait_bar(&redempty[rs], rphase ^ 1u);
     float *rbuf = reinterpret_cast<float *>(smem + p.red_off + rs * p.red_stage);
 #pragma unroll 1
     for (int q = 0; q < ns_t; ++q) {
@@ -914,7 +914,10 @@ __global__ void __launch_bounds__(512, 1)
     pos = pos.plus(ns_t, p.nslot);
     __syncwarp();
     if (lane == 0) mbar_arrive(&redfull[rs]);
-    twr.advance_stage();
+    if (++rs == p.nred) {
+      rs = 0;
+      rphase ^= 1u;
+    }
   }
   if (dead && p.err) atomicOr(p.err, 2);
 }
