@@ -1,7 +1,9 @@
 // qmv_api.cu -- the C ABI of libqmv: argument checks, launch planning and
 // kernel dispatch.  Declarations and the contract of every entry point are in
 // include/qmv.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdarg>
 #include <cstdint>
@@ -10,7 +12,10 @@
 #include <mutex>
 #include <string>
 
+#include <cuda_fp16.h>
+
 #include "qmv.h"
+#include "qmv_mma.cuh"
 #include "qmv_stream.cuh"
 
 namespace {
@@ -59,6 +64,11 @@ struct DeviceInfo {
   int smem_optin = 0;
 };
 constexpr int kMaxDevices = 64;
+#ifndef QMV_MMA_MIN_ROWS
+#define QMV_MMA_MIN_ROWS 3
+#endif
+// fewest activation rows that go to the tensor-core path
+constexpr int kMmaMinRows = QMV_MMA_MIN_ROWS;
 DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 
@@ -280,6 +290,138 @@ int launch(const Plan &pl, int bits, cudaStream_t stream) {
 
 void init_params(qmvk::StreamParams &p) { std::memset(&p, 0, sizeof p); }
 
+// ---------------------------------------------------------------------------
+// Batched rows on the tensor cores (qmv_mma.cuh): up to 16 activation rows
+// share one read of the weights.  2-, 4- and 8-bit codes; K a multiple of
+// one stage row (1024 / bits codes); group sizes 32, 64, 128.
+// ---------------------------------------------------------------------------
+// (K / gs) % 8 == 0 makes the scale / bias row stride a multiple of 16 bytes
+// (a tensor-copy rule).
+bool mma_path(int M, int K, int bits, int gs) {
+  if (!(bits == 2 || bits == 4 || bits == 8)) return false;
+  if (!(gs == 32 || gs == 64 || gs == 128)) return false;
+  return M >= kMmaMinRows && M <= qmvk::kMmaCols && K % (1024 / bits) == 0 &&
+         (K / gs) % 8 == 0;
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link to
+// the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A 2-D row-major tensor [rows][cols] of `esize`-byte elements with row
+// stride `stride` bytes, copied in boxes of [box_rows][box_cols].
+int encode_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, uint64_t cols,
+              uint64_t rows, uint64_t stride, uint32_t box_cols, uint32_t box_rows,
+              CUtensorMapSwizzle swz, CUtensorMapL2promotion l2) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(QMV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, type, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, l2,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QMV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return 0;
+}
+
+template <int BITS, int GS>
+int launch_mma_t(qmvk::MmaParams &mp, int grid, DeviceInfo *dev, cudaStream_t stream) {
+  using ST = qmvk::MmaStage<BITS>;
+  auto kern = qmvk::qmv_mma_kernel<BITS, GS>;
+  mp.stage_bytes = ST::bytes(mp.M);
+  const int room = dev->smem_optin - static_cast<int>(qmvk::MmaSmem::w_off) - 1024;
+  int nst = room / static_cast<int>(mp.stage_bytes);
+  if (nst > qmvk::kMmaMaxStages) nst = qmvk::kMmaMaxStages;
+  if (nst < 2) return fail(QMV_ERR_UNSUPPORTED, "tensor-core path: shared memory too small");
+  mp.nst = nst;
+  const int smem = static_cast<int>(qmvk::MmaSmem::w_off + 1024 + nst * mp.stage_bytes);
+  // tensor maps: codes [N][row_bytes] u8, scales / biases [N][G] u16,
+  // x [M][K] u16
+  CUtensorMap tw, ts, tb, tx;
+  int rc;
+  if ((rc = encode_2d(&tw, mp.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, mp.row_bytes, mp.N, mp.row_bytes,
+                      128, qmvk::kMmaRows, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B)))
+    return rc;
+  if ((rc = encode_2d(&ts, mp.s, CU_TENSOR_MAP_DATA_TYPE_UINT16, mp.G, mp.N, 2ull * mp.G,
+                      qmvk::kMmaWinGroups, qmvk::kMmaRows, CU_TENSOR_MAP_SWIZZLE_32B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B)))
+    return rc;
+  if ((rc = encode_2d(&tb, mp.b, CU_TENSOR_MAP_DATA_TYPE_UINT16, mp.G, mp.N, 2ull * mp.G,
+                      qmvk::kMmaWinGroups, qmvk::kMmaRows, CU_TENSOR_MAP_SWIZZLE_32B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B)))
+    return rc;
+  if ((rc = encode_2d(&tx, mp.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, mp.K, mp.M, 2ull * mp.K,
+                      qmvk::mma_x_slice<BITS>(), mp.M, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B)))
+    return rc;
+  int d = 0;
+  cudaGetDevice(&d);
+  static int granted[kMaxDevices] = {};
+  if (smem > granted[d]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         dev->smem_optin);
+    if (e != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    granted[d] = dev->smem_optin;
+  }
+  kern<<<grid, qmvk::mma_threads<BITS>(), smem, stream>>>(tw, ts, tb, tx, mp);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+template <int BITS>
+int launch_mma_b(qmvk::MmaParams &mp, int gs, int grid, DeviceInfo *dev, cudaStream_t stream) {
+  switch (gs) {
+    case 32: return launch_mma_t<BITS, 32>(mp, grid, dev, stream);
+    case 64: return launch_mma_t<BITS, 64>(mp, grid, dev, stream);
+    case 128: return launch_mma_t<BITS, 128>(mp, grid, dev, stream);
+    default: return fail(QMV_ERR_UNSUPPORTED, "group_size=%d on the tensor-core path", gs);
+  }
+}
+
+int launch_mma(const void *x, const uint32_t *w, const void *scales,
+               const void *biases, void *y, int M, int N, int K, int bits, int gs,
+               DeviceInfo *dev, cudaStream_t stream) {
+  qmvk::MmaParams mp;
+  std::memset(&mp, 0, sizeof mp);
+  mp.w = reinterpret_cast<const uint8_t *>(w);
+  mp.s = static_cast<const uint16_t *>(scales);
+  mp.b = static_cast<const uint16_t *>(biases);
+  mp.x = static_cast<const uint16_t *>(x);
+  mp.y = static_cast<uint16_t *>(y);
+  mp.M = M;
+  mp.N = N;
+  mp.K = K;
+  mp.G = K / gs;
+  mp.row_bytes = static_cast<uint32_t>(static_cast<long long>(K) * bits / 8);
+  mp.ntiles = (N + qmvk::kMmaRows - 1) / qmvk::kMmaRows;
+  mp.nstage = K / (1024 / bits);
+  const int grid = mp.ntiles < dev->sms ? mp.ntiles : dev->sms;
+  switch (bits) {
+    case 2: return launch_mma_b<2>(mp, gs, grid, dev, stream);
+    case 4: return launch_mma_b<4>(mp, gs, grid, dev, stream);
+    case 8: return launch_mma_b<8>(mp, gs, grid, dev, stream);
+    default: return fail(QMV_ERR_UNSUPPORTED, "bits=%d on the tensor-core path", bits);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -301,6 +443,9 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
     return fail(QMV_ERR_ALIGN, "qmv: buffers must be 16-byte aligned");
   DeviceInfo *dev;
   if ((rc = device_info(&dev))) return rc;
+  if (mma_path(M, K, bits, group_size))
+    return launch_mma(x, w, scales, biases, y, M, N, K, bits, group_size, dev,
+                      static_cast<cudaStream_t>(stream));
   Plan pl;
   init_params(pl.p);
   qmvk::StreamParams &p = pl.p;

@@ -103,3 +103,38 @@ def test_qmv_many_chunks_tiny_rows():
     y = run_qmv(x, w, s, b, M, N, K, bits, gs)
     y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, nthreads=8)
     check(y, y_ref, a_ref, "qmv many chunks")
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_qmv_batched_rows_small(bits, gs):
+    # several activation rows (the tensor-core path for 2/4/8-bit codes):
+    # three 128-row tiles with a ragged last one, several K stages
+    for M in (3, 5, 16):
+        N, K = 300, 2048
+        x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=7000 + 31 * M + bits + gs)
+        y = run_qmv(x, w, s, b, M, N, K, bits, gs)
+        y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs)
+        check(y, y_ref, a_ref, f"batched rows M={M} bits={bits} gs={gs}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 7, 8, 12, 16])
+def test_qmv_batched_rows_counts(M):
+    # every activation-row count up to 16 at one shape, a single K stage
+    bits, gs, N, K = 4, 32, 129, 256
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=7500 + M)
+    y = run_qmv(x, w, s, b, M, N, K, bits, gs)
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs)
+    check(y, y_ref, a_ref, f"batched rows M={M}")
+
+
+def test_qmv_batched_many_tiles_per_cta():
+    # more than two 128-row tiles per CTA on any current GPU (the accumulator
+    # halves and the stage ring are both reused), ragged last tile; oracle on
+    # sampled rows plus the last rows
+    M, N, K, bits, gs = 6, 3 * 160 * 128 + 77, 2048, 4, 64
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=7777)
+    y = run_qmv(x, w, s, b, M, N, K, bits, gs)
+    rows = np.unique(np.concatenate([sample_rows(N, 300, seed=5), np.arange(N - 80, N)])).astype(np.int32)
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, rows=rows, nthreads=8)
+    check(y[:, rows], y_ref, a_ref, "batched many tiles")
