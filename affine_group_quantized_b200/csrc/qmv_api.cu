@@ -413,6 +413,11 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   mp.row_bytes = static_cast<uint32_t>(static_cast<long long>(K) * bits / 8);
   mp.ntiles = (N + qmvk::kMmaRows - 1) / qmvk::kMmaRows;
   mp.nstage = K / (1024 / bits);
+  mp.k_magic = 0x64006400u;
+  for (int i = 0; i < 3; ++i) {
+    const uint32_t a = 0x8000u | (static_cast<uint32_t>(25 - (2 * i + 2)) << 10);
+    mp.k_add[i] = a | (a << 16);
+  }
   const int grid = mp.ntiles < dev->sms ? mp.ntiles : dev->sms;
   switch (bits) {
     case 2: return launch_mma_b<2>(mp, gs, grid, dev, stream);

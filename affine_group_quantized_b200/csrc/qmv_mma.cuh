@@ -54,6 +54,10 @@ struct MmaParams {
   int nstage;            // K / (codes per stage row)
   int nst;               // stages in the shared-memory ring
   uint32_t stage_bytes;  // bytes of one stage (depends on M), 1024-aligned
+  // dequant constants, passed in so that they live in registers for the
+  // whole loop (an FMA or a 3-input logic op takes one immediate only)
+  uint32_t k_magic;      // 0x64006400: fp16 1024 in each half
+  uint32_t k_add[3];     // -1024 * 2^-SH in each half, SH = 2, 4, 6
 };
 
 constexpr int kMmaRows = 128;    // weight rows per tile (the MMA's M)
@@ -62,7 +66,14 @@ constexpr int kMmaCols = 16;     // x rows per MMA (the MMA's N)
 // fp16 A operands in flight in tensor memory (64 columns each, one per MMA
 // chunk); the MMAs of a chunk complete well after they are issued, so the
 // dequant warps run ahead
-constexpr int kMmaAbufs = 7;
+#ifndef QMV_MMA_NACC
+#define QMV_MMA_NACC 4
+#endif
+// Independent accumulators per tile: the eight K = 16 MMAs of a chunk go
+// round-robin to kMmaNacc accumulators (summed in the epilogue), so that
+// consecutive MMAs do not wait on each other's result.
+constexpr int kMmaNacc = QMV_MMA_NACC;
+constexpr int kMmaAbufs = (512 - 2 * kMmaNacc * 16) / 64 < 7 ? (512 - 2 * kMmaNacc * 16) / 64 : 7;
 constexpr uint32_t kMmaACols = kMmaKC / 2;             // 32-bit columns of one A
 constexpr uint32_t kMmaDCol = kMmaAbufs * kMmaACols;   // first accumulator column
 constexpr uint32_t kMmaTmemCols = 512;                 // allocation (power of two)
@@ -300,15 +311,15 @@ __device__ __forceinline__ __half2 h2_bits(uint32_t v) {
 __device__ __forceinline__ uint32_t h2_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 
 template <int SH>
-__device__ __forceinline__ uint32_t code_fma(uint32_t h, __half2 s2, __half2 b2) {
+__device__ __forceinline__ uint32_t code_fma(uint32_t h, __half2 s2, __half2 b2,
+                                             const uint32_t (&kadd)[3]) {
   __half2 q;
   if constexpr (SH == 0) {
     q = __hsub2(h2_bits(h), h2_bits(0x64006400u));
   } else {
-    // 2^-SH and -1024 * 2^-SH as fp16 pairs
+    // h * 2^-SH + (-1024 * 2^-SH)
     constexpr uint32_t m = static_cast<uint32_t>(15 - SH) << 10;
-    constexpr uint32_t a = 0x8000u | (static_cast<uint32_t>(25 - SH) << 10);
-    q = __hfma2(h2_bits(h), h2_bits(m | (m << 16)), h2_bits(a | (a << 16)));
+    q = __hfma2(h2_bits(h), h2_bits(m | (m << 16)), h2_bits(kadd[SH / 2 - 1]));
   }
   return h2_u32(__hfma2(q, s2, b2));
 }
@@ -328,29 +339,29 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // the upper half of every 16-bit lane), so most of the work is on the
 // fp16 pipe rather than the half-rate integer pipe.
 template <int BITS>
-__device__ __forceinline__ void dequant_word(uint32_t w, __half2 s2, __half2 b2,
+__device__ __forceinline__ void dequant_word(uint32_t w, __half2 s2, __half2 b2, uint32_t kmagic,
+                                             const uint32_t (&kadd)[3],
                                              uint32_t (&h)[16 / BITS]) {
-  constexpr uint32_t kMagic = 0x64006400u;
   if constexpr (BITS == 8) {
     // bytes (0, 2) and (1, 3) under a 0x64 high byte
-    h[0] = code_fma<0>(prmt(w, 0x64646464u, 0x4240u), s2, b2);
-    h[1] = code_fma<0>(prmt(w, 0x64646464u, 0x4341u), s2, b2);
+    h[0] = code_fma<0>(prmt(w, kmagic, 0x7250u), s2, b2, kadd);
+    h[1] = code_fma<0>(prmt(w, kmagic, 0x7351u), s2, b2, kadd);
   } else if constexpr (BITS == 4) {
     const uint32_t v = w >> 8;
-    h[0] = code_fma<0>((w & 0x000f000fu) | kMagic, s2, b2);
-    h[1] = code_fma<4>((w & 0x00f000f0u) | kMagic, s2, b2);
-    h[2] = code_fma<0>((v & 0x000f000fu) | kMagic, s2, b2);
-    h[3] = code_fma<4>((v & 0x00f000f0u) | kMagic, s2, b2);
+    h[0] = code_fma<0>((w & 0x000f000fu) | kmagic, s2, b2, kadd);
+    h[1] = code_fma<4>((w & 0x00f000f0u) | kmagic, s2, b2, kadd);
+    h[2] = code_fma<0>((v & 0x000f000fu) | kmagic, s2, b2, kadd);
+    h[3] = code_fma<4>((v & 0x00f000f0u) | kmagic, s2, b2, kadd);
   } else {
     const uint32_t v = w >> 8;
-    h[0] = code_fma<0>((w & 0x00030003u) | kMagic, s2, b2);
-    h[1] = code_fma<2>((w & 0x000c000cu) | kMagic, s2, b2);
-    h[2] = code_fma<4>((w & 0x00300030u) | kMagic, s2, b2);
-    h[3] = code_fma<6>((w & 0x00c000c0u) | kMagic, s2, b2);
-    h[4] = code_fma<0>((v & 0x00030003u) | kMagic, s2, b2);
-    h[5] = code_fma<2>((v & 0x000c000cu) | kMagic, s2, b2);
-    h[6] = code_fma<4>((v & 0x00300030u) | kMagic, s2, b2);
-    h[7] = code_fma<6>((v & 0x00c000c0u) | kMagic, s2, b2);
+    h[0] = code_fma<0>((w & 0x00030003u) | kmagic, s2, b2, kadd);
+    h[1] = code_fma<2>((w & 0x000c000cu) | kmagic, s2, b2, kadd);
+    h[2] = code_fma<4>((w & 0x00300030u) | kmagic, s2, b2, kadd);
+    h[3] = code_fma<6>((w & 0x00c000c0u) | kmagic, s2, b2, kadd);
+    h[4] = code_fma<0>((v & 0x00030003u) | kmagic, s2, b2, kadd);
+    h[5] = code_fma<2>((v & 0x000c000cu) | kmagic, s2, b2, kadd);
+    h[6] = code_fma<4>((v & 0x00300030u) | kmagic, s2, b2, kadd);
+    h[7] = code_fma<6>((v & 0x00c000c0u) | kmagic, s2, b2, kadd);
   }
 }
 
@@ -558,22 +569,32 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
     int tl = 0;  // tiles done (accumulator buffer position)
     bool dead = false;
     const int nchunks = p.nstage * CPS;
+    const uint64_t bdesc0 = mma_smem_desc(base + MmaSmem::b_off);
     for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tl) {
       const int db = tl & 1;
       const uint32_t dph = static_cast<uint32_t>((tl >> 1) & 1);
       if (tl >= 2 && !dead && !mbar_wait_sleep(&dempty[db], dph ^ 1u)) dead = true;
       tc_fence_after();
-      const uint32_t tmem_d = tmem_base + kMmaDCol + db * kMmaCols;
+      const uint32_t tmem_d = tmem_base + kMmaDCol + db * (kMmaNacc * kMmaCols);
       for (int c = 0; c < nchunks; ++c) {
         if (!dead && !mbar_wait_sleep(&abfull[ap.idx], ap.phase)) dead = true;
         tc_fence_after();
         if (lane == 0) {
+          // descriptors advance by whole 16-byte units inside the start
+          // address field (shared addresses stay below 2^18)
           const uint32_t a0 = tmem_base + ap.idx * kMmaACols;
-          const uint32_t b0 = base + MmaSmem::b_off + ap.idx * kMmaBBytes;
+          const uint64_t d0 = bdesc0 + static_cast<uint64_t>(ap.idx * (kMmaBBytes >> 4));
+          if (c == 0) {
 #pragma unroll
-          for (int j = 0; j < kMmaKC / 16; ++j)
-            mma_f16_ta(tmem_d, a0 + j * 8, mma_smem_desc(b0 + j * 2 * kMmaLBO),
-                       (c > 0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < kMmaKC / 16; ++j)
+              mma_f16_ta(tmem_d + (j % kMmaNacc) * kMmaCols, a0 + j * 8,
+                         d0 + static_cast<uint64_t>(j * (2 * kMmaLBO >> 4)), j >= kMmaNacc ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < kMmaKC / 16; ++j)
+              mma_f16_ta(tmem_d + (j % kMmaNacc) * kMmaCols, a0 + j * 8,
+                         d0 + static_cast<uint64_t>(j * (2 * kMmaLBO >> 4)), 1u);
+          }
           mma_commit(&abempty[ap.idx]);
           if (c == nchunks - 1) mma_commit(&dfull[db]);
         }
@@ -625,142 +646,179 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
       xq[ui] = kg % GPS;
       xm[ui] = xmul[m];
     }
+    const uint32_t kmagic = p.k_magic;
+    const uint32_t kadd[3] = {p.k_add[0], p.k_add[1], p.k_add[2]};
     RingPos sp, ap;
     // this thread's first operand buffer: chunk cc of the first stage
     for (int i = 0; i < cc; ++i) ap.next(NAB);
     long long kc = cc;  // MMA chunk count of this thread's chunk
-    int tl = 0;
     bool dead = false;
-    for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tl) {
-      for (int c = 0; c < p.nstage; ++c) {
-        if (!dead && !mbar_wait(&wfull[sp.idx], sp.phase)) dead = true;
-        const uint32_t stg = ring + sp.idx * sbytes;
-        uint32_t wd[QW];
+    const bool x_warp = (xw & ~31) < nunits;  // this warp writes B units
+    // What a stage leaves in registers: the part's words, its groups'
+    // scale / bias pairs and the x spans behind this thread's B units.
+    struct Regs {
+      uint32_t wd[QW];
+      __half2 s2[NG], b2[NG];
+      uint4 xv[UPT][SPAN / 8];
+    };
+    // Wait for stage c of the ring, read this thread's share of it, then
+    // hand the stage back to the producer.
+    auto load = [&](Regs &R, int c) {
+      if (!dead && !mbar_wait(&wfull[sp.idx], sp.phase)) dead = true;
+      const uint32_t stg = ring + sp.idx * sbytes;
 #pragma unroll
-        for (int i = 0; i < QW / 4; ++i)
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-                       : "=r"(wd[4 * i]), "=r"(wd[4 * i + 1]), "=r"(wd[4 * i + 2]),
-                         "=r"(wd[4 * i + 3])
-                       : "r"(stg + woff[i]));
-        // scale / bias of each group the part touches, as fp16 pairs: NG
-        // groups from window index gh (a multiple of NG, so one aligned
-        // load); 32-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 4) % 2)
-        const int gh = ((c * (SC / GS)) & 7) + gpart;
-        const uint32_t wo = wrow + ((((2 * gh) >> 4) ^ wswz) << 4) + ((2 * gh) & 15);
-        uint32_t sv[(NG + 1) / 2], bv[(NG + 1) / 2];
-        lds_groups<NG>(stg + ST::s_off + wo, sv);
-        lds_groups<NG>(stg + ST::b_off + wo, bv);
-        uint4 xv[UPT][SPAN / 8];
+      for (int i = 0; i < QW / 4; ++i)
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                     : "=r"(R.wd[4 * i]), "=r"(R.wd[4 * i + 1]), "=r"(R.wd[4 * i + 2]),
+                       "=r"(R.wd[4 * i + 3])
+                     : "r"(stg + woff[i]));
+      // NG groups from window index gh (a multiple of NG, so one aligned
+      // load); 32-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 4) % 2)
+      const int gh = ((c * (SC / GS)) & 7) + gpart;
+      const uint32_t wo = wrow + ((((2 * gh) >> 4) ^ wswz) << 4) + ((2 * gh) & 15);
+      uint32_t sv[(NG + 1) / 2], bv[(NG + 1) / 2];
+      lds_groups<NG>(stg + ST::s_off + wo, sv);
+      lds_groups<NG>(stg + ST::b_off + wo, bv);
 #pragma unroll
-        for (int ui = 0; ui < UPT; ++ui) {
-          if (xw + ui * TW < nunits) {
+      for (int ui = 0; ui < UPT; ++ui) {
+        if (xw + ui * TW < nunits) {
 #pragma unroll
-            for (int i = 0; i < SPAN / 8; ++i)
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-                           : "=r"(xv[ui][i].x), "=r"(xv[ui][i].y), "=r"(xv[ui][i].z),
-                             "=r"(xv[ui][i].w)
-                           : "r"(stg + xsrc[ui] + 16 * i));
-          }
+          for (int i = 0; i < SPAN / 8; ++i)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                         : "=r"(R.xv[ui][i].x), "=r"(R.xv[ui][i].y), "=r"(R.xv[ui][i].z),
+                           "=r"(R.xv[ui][i].w)
+                         : "r"(stg + xsrc[ui] + 16 * i));
         }
-        __half2 s2[NG], b2[NG];
+      }
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          s2[g] = h2_bits(bf16_to_half2_dup((sv[g / 2] >> (16 * (g % 2))) & 0xffffu));
-          b2[g] = h2_bits(bf16_to_half2_dup((bv[g / 2] >> (16 * (g % 2))) & 0xffffu));
+      for (int g = 0; g < NG; ++g) {
+        R.s2[g] = h2_bits(bf16_to_half2_dup((sv[g / 2] >> (16 * (g % 2))) & 0xffffu));
+        R.b2[g] = h2_bits(bf16_to_half2_dup((bv[g / 2] >> (16 * (g % 2))) & 0xffffu));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[sp.idx]);
+      sp.next(nst);
+    };
+    // Stage (t, c) from registers R: fp16 weights into tensor memory, the x
+    // units into the B buffer; the next stage is read into N while the
+    // stores drain, then the chunk is handed to the MMA warp.
+    int t = blockIdx.x, c = 0, tl = 0;
+    auto step = [&](Regs &R, Regs &N) {
+      // the operand buffer must be free: its previous MMAs have completed
+      if (kc >= NAB && !dead && !mbar_wait(&abempty[ap.idx], ap.phase ^ 1u)) dead = true;
+      tc_fence_after();
+      uint32_t av[NV];
+#pragma unroll
+      for (int s = 0; s < NSP; ++s) {
+        const int g = (QC >= GS) ? (s * SPAN) / GS : 0;  // compile time
+#pragma unroll
+        for (int wi = 0; wi < WPS; ++wi) {
+          uint32_t hw[16 / BITS];
+          dequant_word<BITS>(R.wd[s * WPS + wi], R.s2[g], R.b2[g], kmagic, kadd, hw);
+#pragma unroll
+          for (int j = 0; j < 16 / BITS; ++j) av[(s * WPS + wi) * (16 / BITS) + j] = hw[j];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&wempty[sp.idx]);
-        sp.next(nst);
-        // the operand buffer must be free: its previous MMAs have completed
-        if (kc >= NAB && !dead && !mbar_wait(&abempty[ap.idx], ap.phase ^ 1u)) dead = true;
-        tc_fence_after();
-        uint32_t av[NV];
-#pragma unroll
-        for (int s = 0; s < NSP; ++s) {
-          const int g = (QC >= GS) ? (s * SPAN) / GS : 0;  // compile time
-#pragma unroll
-          for (int wi = 0; wi < WPS; ++wi) {
-            uint32_t hw[16 / BITS];
-            dequant_word<BITS>(wd[s * WPS + wi], s2[g], b2[g], hw);
-#pragma unroll
-            for (int j = 0; j < 16 / BITS; ++j) av[(s * WPS + wi) * (16 / BITS) + j] = hw[j];
-          }
-        }
-        const uint32_t ta = ta0 + ap.idx * kMmaACols;
+      }
+      const uint32_t ta = ta0 + ap.idx * kMmaACols;
 #ifndef QMV_MMA_ST
 #define QMV_MMA_ST 32
 #endif
-        constexpr int STC = QMV_MMA_ST < NV ? QMV_MMA_ST : NV;  // columns per store
-        if constexpr (STC == 8) {
+      constexpr int STC = QMV_MMA_ST < NV ? QMV_MMA_ST : NV;  // columns per store
+      if constexpr (STC == 8) {
 #pragma unroll
-          for (int i = 0; i < NV / 8; ++i) tmem_st8(ta + 8 * i, &av[8 * i]);
-        } else if constexpr (STC == 16) {
+        for (int i = 0; i < NV / 8; ++i) tmem_st8(ta + 8 * i, &av[8 * i]);
+      } else if constexpr (STC == 16) {
 #pragma unroll
-          for (int i = 0; i < NV / 16; ++i)
-            tmem_st16(ta + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&av[16 * i]));
-        } else {
+        for (int i = 0; i < NV / 16; ++i)
+          tmem_st16(ta + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&av[16 * i]));
+      } else {
 #pragma unroll
-          for (int i = 0; i < NV / 32; ++i)
-            tmem_st32(ta + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&av[32 * i]));
+        for (int i = 0; i < NV / 32; ++i)
+          tmem_st32(ta + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&av[32 * i]));
+      }
+      const uint32_t bbuf = base + ap.idx * kMmaBBytes;
+#pragma unroll
+      for (int ui = 0; ui < UPT; ++ui) {
+        if (xw + ui * TW < nunits) {
+          float xs[SPAN];
+#pragma unroll
+          for (int i = 0; i < SPAN / 8; ++i) {
+            const uint32_t qq[4] = {R.xv[ui][i].x, R.xv[ui][i].y, R.xv[ui][i].z, R.xv[ui][i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              xs[8 * i + 2 * j] = __uint_as_float(qq[j] << 16) * xm[ui];
+              xs[8 * i + 2 * j + 1] = __uint_as_float(qq[j] & 0xffff0000u) * xm[ui];
+            }
+          }
+          uint32_t hv[4];
+          if (GPS == 1 || xq[ui] == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              hv[i] = pack_half2(xs[mma_k_of(BITS, 0, 2 * i)], xs[mma_k_of(BITS, 0, 2 * i + 1)]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              hv[i] = pack_half2(xs[mma_k_of(BITS, 1, 2 * i)], xs[mma_k_of(BITS, 1, 2 * i + 1)]);
+          }
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(bbuf + xdst[ui]),
+                       "r"(hv[0]), "r"(hv[1]), "r"(hv[2]), "r"(hv[3])
+                       : "memory");
         }
-        const uint32_t bbuf = base + ap.idx * kMmaBBytes;
+      }
+      // the next stage of this CTA's walk
+      const int tc = t, cc_last = (c == p.nstage - 1);
+      if (++c == p.nstage) {
+        c = 0;
+        t += gridDim.x;
+      }
+      if (t < p.ntiles) load(N, c);
+      tmem_wait_st();
+      // make the tensor-memory stores, and the B units' generic-proxy
+      // shared stores, visible to the MMA
+      if (x_warp) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&abfull[ap.idx]);
+      for (int i = 0; i < CPS; ++i) ap.next(NAB);
+      kc += CPS;
+      // ---- epilogue of tile tc after its last stage: warps 0..3 read the
+      // accumulator ----
+      if (cc_last) {
+        if (warp < 4) {
+          const int db = tl & 1;
+          const uint32_t dph = static_cast<uint32_t>((tl >> 1) & 1);
+          if (!dead && !mbar_wait(&dfull[db], dph)) dead = true;
+          tc_fence_after();
+          float d[16];
+          const uint32_t dcol = tmem_base + (static_cast<uint32_t>(32 * warp) << 16) + kMmaDCol +
+                                db * (kMmaNacc * kMmaCols);
+          tmem_ld16(dcol, d);
 #pragma unroll
-        for (int ui = 0; ui < UPT; ++ui) {
-          if (xw + ui * TW < nunits) {
-            float xs[SPAN];
+          for (int a = 1; a < kMmaNacc; ++a) {
+            float e[16];
+            tmem_ld16(dcol + a * kMmaCols, e);
 #pragma unroll
-            for (int i = 0; i < SPAN / 8; ++i) {
-              const uint32_t qq[4] = {xv[ui][i].x, xv[ui][i].y, xv[ui][i].z, xv[ui][i].w};
+            for (int m = 0; m < 16; ++m) d[m] += e[m];
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dempty[db]);
+          const int row = tc * kMmaRows + 32 * warp + lane;
+          if (row < p.N) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                xs[8 * i + 2 * j] = __uint_as_float(qq[j] << 16) * xm[ui];
-                xs[8 * i + 2 * j + 1] = __uint_as_float(qq[j] & 0xffff0000u) * xm[ui];
-              }
-            }
-            uint32_t hv[4];
-            if (GPS == 1 || xq[ui] == 0) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                hv[i] = pack_half2(xs[mma_k_of(BITS, 0, 2 * i)], xs[mma_k_of(BITS, 0, 2 * i + 1)]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                hv[i] = pack_half2(xs[mma_k_of(BITS, 1, 2 * i)], xs[mma_k_of(BITS, 1, 2 * i + 1)]);
-            }
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(bbuf + xdst[ui]),
-                         "r"(hv[0]), "r"(hv[1]), "r"(hv[2]), "r"(hv[3])
-                         : "memory");
+            for (int m = 0; m < kMmaCols; ++m)
+              if (m < p.M) p.y[static_cast<size_t>(m) * p.N + row] = f32_to_bf16(d[m] * xinv[m]);
           }
         }
-        tmem_wait_st();
-        // make the tensor-memory stores and the generic-proxy shared stores
-        // visible to the MMA
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&abfull[ap.idx]);
-        for (int i = 0; i < CPS; ++i) ap.next(NAB);
-        kc += CPS;
+        ++tl;
       }
-      // ---- epilogue of tile t: warps 0..3 read the accumulator ----
-      if (warp < 4) {
-        const int db = tl & 1;
-        const uint32_t dph = static_cast<uint32_t>((tl >> 1) & 1);
-        if (!dead && !mbar_wait(&dfull[db], dph)) dead = true;
-        tc_fence_after();
-        float d[16];
-        tmem_ld16(tmem_base + (static_cast<uint32_t>(32 * warp) << 16) + kMmaDCol + db * kMmaCols,
-                  d);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[db]);
-        const int row = t * kMmaRows + 32 * warp + lane;
-        if (row < p.N) {
-#pragma unroll
-          for (int m = 0; m < kMmaCols; ++m)
-            if (m < p.M) p.y[static_cast<size_t>(m) * p.N + row] = f32_to_bf16(d[m] * xinv[m]);
-        }
-      }
+    };
+    Regs A, B;
+    if (t < p.ntiles) load(A, 0);
+    while (t < p.ntiles) {
+      step(A, B);
+      if (t >= p.ntiles) break;
+      step(B, A);
     }
     if (dead && p.err && lane == 0) atomicOr(p.err, 2);
   }
