@@ -338,6 +338,41 @@ int encode_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, uint6
   return 0;
 }
 
+// Scratch of the tensor-core path, one per device, made on first use and
+// grown when a call needs more: the partial-sum slots (two per CTA) and one
+// arrival counter per tile (zero between launches: the last arrival resets
+// it).  Calls that use it on one device are expected in stream order.
+struct MmaScratch {
+  float *part = nullptr;
+  int *cnt = nullptr;
+  int cnt_len = 0;
+};
+MmaScratch g_mma_scratch[kMaxDevices];
+std::mutex g_mma_scratch_mu;
+
+int mma_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
+  std::lock_guard<std::mutex> lock(g_mma_scratch_mu);
+  MmaScratch &s = g_mma_scratch[dev_id];
+  if (!s.part) {
+    const size_t bytes = static_cast<size_t>(sms) * 2 * qmvk::kMmaCols * qmvk::kMmaRows * 4;
+    if (cudaMalloc(&s.part, bytes) != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "tensor-core path: cannot allocate %zu bytes of scratch", bytes);
+  }
+  if (s.cnt_len < ntiles) {
+    int n = s.cnt_len ? s.cnt_len : 1024;
+    while (n < ntiles) n *= 2;
+    int *c = nullptr;
+    if (cudaMalloc(&c, static_cast<size_t>(n) * 4) != cudaSuccess ||
+        cudaMemset(c, 0, static_cast<size_t>(n) * 4) != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "tensor-core path: cannot allocate the tile counters");
+    if (s.cnt) cudaFree(s.cnt);  // waits for the launches that use it
+    s.cnt = c;
+    s.cnt_len = n;
+  }
+  *out = &s;
+  return 0;
+}
+
 template <int BITS, int GS>
 int launch_mma_t(qmvk::MmaParams &mp, int grid, DeviceInfo *dev, cudaStream_t stream) {
   using ST = qmvk::MmaStage<BITS>;
@@ -413,12 +448,23 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   mp.row_bytes = static_cast<uint32_t>(static_cast<long long>(K) * bits / 8);
   mp.ntiles = (N + qmvk::kMmaRows - 1) / qmvk::kMmaRows;
   mp.nstage = K / (1024 / bits);
+  mp.nsteps = static_cast<long long>(mp.ntiles) * mp.nstage;
   mp.k_magic = 0x64006400u;
   for (int i = 0; i < 3; ++i) {
     const uint32_t a = 0x8000u | (static_cast<uint32_t>(25 - (2 * i + 2)) << 10);
     mp.k_add[i] = a | (a << 16);
   }
-  const int grid = mp.ntiles < dev->sms ? mp.ntiles : dev->sms;
+  // one whole tile per CTA when the tiles fit the SMs; otherwise every SM
+  // takes an equal share of the (tile, stage) steps (tiles cut between CTAs
+  // are added up through the scratch slots)
+  const int grid = mp.ntiles <= dev->sms ? mp.ntiles : dev->sms;
+  int d = 0;
+  cudaGetDevice(&d);
+  MmaScratch *sc = nullptr;
+  int rc;
+  if ((rc = mma_scratch(d, dev->sms, mp.ntiles, &sc))) return rc;
+  mp.part = sc->part;
+  mp.cnt = sc->cnt;
   switch (bits) {
     case 2: return launch_mma_b<2>(mp, gs, grid, dev, stream);
     case 4: return launch_mma_b<4>(mp, gs, grid, dev, stream);

@@ -52,6 +52,16 @@ struct MmaParams {
   uint32_t row_bytes;    // K * bits / 8
   int ntiles;            // ceil(N / 128)
   int nstage;            // K / (codes per stage row)
+  // Stream-K walk: the ntiles * nstage (tile, stage) steps, tile-major, are
+  // cut into gridDim.x equal contiguous ranges, one per CTA (with as many
+  // CTAs as tiles, every range is one whole tile).  A tile cut by
+  // a range boundary leaves fp32 partial sums in `part` (two slots per CTA:
+  // its first and its last segment, 16 x 128 floats each); the last CTA to
+  // finish the tile (counted in cnt[tile], reset to 0 afterwards) adds the
+  // parts in CTA order and stores y.
+  long long nsteps;      // ntiles * nstage
+  float *part;           // [gridDim.x][2][16][128]
+  int *cnt;              // [ntiles], zero between launches
   int nst;               // stages in the shared-memory ring
   uint32_t stage_bytes;  // bytes of one stage (depends on M), 1024-aligned
   // dequant constants, passed in so that they live in registers for the
@@ -105,6 +115,7 @@ __host__ __device__ constexpr int mma_x_slice() { return mma_stage_codes<BITS>()
 // A stage: the packed rows [128][128 B], the scale and bias windows
 // [128][32 B], then the x slices [slice][M][slice codes] (bf16).
 constexpr int kMmaMaxStages = 16;
+
 template <int BITS>
 struct MmaStage {
   static constexpr uint32_t s_off = kMmaRows * 128;
@@ -127,7 +138,8 @@ struct MmaSmem {
   static constexpr uint32_t xinv_off = bar_off + nbar * 8;
   static constexpr uint32_t tmem_off = xinv_off + kMmaCols * 4;
   static constexpr uint32_t xmul_off = tmem_off + 16;
-  static constexpr uint32_t w_off = (xmul_off + kMmaCols * 4 + 1023) / 1024 * 1024;
+  static constexpr uint32_t flag_off = xmul_off + kMmaCols * 4;  // "this CTA ends the tile"
+  static constexpr uint32_t w_off = (flag_off + 16 + 1023) / 1024 * 1024;
 };
 
 // ---------------------------------------------------------------------------
@@ -413,6 +425,14 @@ __host__ __device__ constexpr int mma_warps_per_chunk() { return 4 * (kMmaKC / m
 template <int BITS>
 __host__ __device__ constexpr int mma_threads() { return (4 * mma_parts<BITS>() + 2) * 32; }
 
+// First step of CTA i's range, and the CTA whose range holds step v.
+__device__ __forceinline__ long long mma_range_start(long long i, long long nsteps, int grid) {
+  return i * nsteps / grid;
+}
+__device__ __forceinline__ int mma_range_of(long long v, long long nsteps, int grid) {
+  return static_cast<int>(((v + 1) * grid - 1) / nsteps);
+}
+
 template <int BITS, int GS>
 __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
     qmv_mma_kernel(const __grid_constant__ CUtensorMap tm_w,
@@ -517,6 +537,8 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
   }
   if (warp < nw) named_sync(1, nw * 32);  // dequant warps only (the multipliers)
   const uint32_t tmem_base = *tmem_slot;
+  const long long v0 = mma_range_start(blockIdx.x, p.nsteps, gridDim.x);
+  const long long v1 = mma_range_start(blockIdx.x + 1, p.nsteps, gridDim.x);
 
   if (warp == nw) {
     // ---------------- producer (one thread) ----------------
@@ -530,9 +552,10 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
       constexpr int XS = mma_x_slice<BITS>();
       const uint32_t tx = ST::tx_bytes(p.M);
       const uint32_t xstep = p.M * ST::x_row;
-      for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
-        const int r0 = t * kMmaRows;
-        for (int c = 0; c < p.nstage; ++c, ++issued) {
+      int t = static_cast<int>(v0 / p.nstage), c = static_cast<int>(v0 % p.nstage);
+      for (long long v = v0; v < v1; ++v, ++issued) {
+        {
+          const int r0 = t * kMmaRows;
           if (issued >= nst && !dead && !mbar_wait_sleep(&wempty[sp.idx], sp.phase ^ 1u))
             dead = true;
           const uint32_t dst = ring + sp.idx * sbytes;
@@ -546,6 +569,10 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
           for (int xs = 0; xs < SC / XS; ++xs)
             tma_load_2d(dst + ST::x_off + xs * xstep, &tm_x, c * SC + xs * XS, 0, bar);
           sp.next(nst);
+        }
+        if (++c == p.nstage) {
+          c = 0;
+          ++t;
         }
       }
       // every copy issued must land before the CTA exits: wait (bounded)
@@ -566,17 +593,24 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
   } else if (warp == nw + 1) {
     // ---------------- MMA warp ----------------
     RingPos ap;  // operand buffer position
-    int tl = 0;  // tiles done (accumulator buffer position)
+    int sidx = 0;  // segments done (accumulator buffer position)
     bool dead = false;
-    const int nchunks = p.nstage * CPS;
     const uint64_t bdesc0 = mma_smem_desc(base + MmaSmem::b_off);
-    for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tl) {
-      const int db = tl & 1;
-      const uint32_t dph = static_cast<uint32_t>((tl >> 1) & 1);
-      if (tl >= 2 && !dead && !mbar_wait_sleep(&dempty[db], dph ^ 1u)) dead = true;
-      tc_fence_after();
-      const uint32_t tmem_d = tmem_base + kMmaDCol + db * (kMmaNacc * kMmaCols);
-      for (int c = 0; c < nchunks; ++c) {
+    int c = static_cast<int>(v0 % p.nstage);
+    bool seg_start = true;
+    uint32_t tmem_d = 0;
+    int db = 0;
+    for (long long v = v0; v < v1; ++v) {
+      if (seg_start) {
+        db = sidx & 1;
+        const uint32_t dph = static_cast<uint32_t>((sidx >> 1) & 1);
+        if (sidx >= 2 && !dead && !mbar_wait_sleep(&dempty[db], dph ^ 1u)) dead = true;
+        tc_fence_after();
+        tmem_d = tmem_base + kMmaDCol + db * (kMmaNacc * kMmaCols);
+      }
+      const bool seg_end = (c == p.nstage - 1) || (v == v1 - 1);
+#pragma unroll 1
+      for (int h = 0; h < CPS; ++h) {
         if (!dead && !mbar_wait_sleep(&abfull[ap.idx], ap.phase)) dead = true;
         tc_fence_after();
         if (lane == 0) {
@@ -584,7 +618,7 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
           // address field (shared addresses stay below 2^18)
           const uint32_t a0 = tmem_base + ap.idx * kMmaACols;
           const uint64_t d0 = bdesc0 + static_cast<uint64_t>(ap.idx * (kMmaBBytes >> 4));
-          if (c == 0) {
+          if (seg_start && h == 0) {
 #pragma unroll
             for (int j = 0; j < kMmaKC / 16; ++j)
               mma_f16_ta(tmem_d + (j % kMmaNacc) * kMmaCols, a0 + j * 8,
@@ -596,11 +630,14 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
                          d0 + static_cast<uint64_t>(j * (2 * kMmaLBO >> 4)), 1u);
           }
           mma_commit(&abempty[ap.idx]);
-          if (c == nchunks - 1) mma_commit(&dfull[db]);
+          if (seg_end && h == CPS - 1) mma_commit(&dfull[db]);
         }
         __syncwarp();
         ap.next(NAB);
       }
+      if (seg_end) ++sidx;
+      seg_start = seg_end;
+      if (++c == p.nstage) c = 0;
     }
     if (dead && p.err && lane == 0) atomicOr(p.err, 2);
   } else {
@@ -702,7 +739,12 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
     // Stage (t, c) from registers R: fp16 weights into tensor memory, the x
     // units into the B buffer; the next stage is read into N while the
     // stores drain, then the chunk is handed to the MMA warp.
-    int t = blockIdx.x, c = 0, tl = 0;
+    // the walk: step v of the CTA's range is stage c of tile t; the current
+    // segment (the range's steps inside one tile) began at stage cseg0
+    long long v = v0;
+    int t = static_cast<int>(v0 / p.nstage), c = static_cast<int>(v0 % p.nstage);
+    int cseg0 = c, sidx = 0;
+    int *tile_flag = reinterpret_cast<int *>(smem + MmaSmem::flag_off);
     auto step = [&](Regs &R, Regs &N) {
       // the operand buffer must be free: its previous MMAs have completed
       if (kc >= NAB && !dead && !mbar_wait(&abempty[ap.idx], ap.phase ^ 1u)) dead = true;
@@ -766,12 +808,16 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
         }
       }
       // the next stage of this CTA's walk
-      const int tc = t, cc_last = (c == p.nstage - 1);
+      const int tc = t;
+      const bool seg_end = (c == p.nstage - 1) || (v == v1 - 1);
+      const bool whole_tile = seg_end && cseg0 == 0 && c == p.nstage - 1;
+      ++v;
       if (++c == p.nstage) {
         c = 0;
-        t += gridDim.x;
+        ++t;
       }
-      if (t < p.ntiles) load(N, c);
+      if (seg_end) cseg0 = c;
+      if (v < v1) load(N, c);
       tmem_wait_st();
       // make the tensor-memory stores, and the B units' generic-proxy
       // shared stores, visible to the MMA
@@ -781,12 +827,11 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
       if (lane == 0) mbar_arrive(&abfull[ap.idx]);
       for (int i = 0; i < CPS; ++i) ap.next(NAB);
       kc += CPS;
-      // ---- epilogue of tile tc after its last stage: warps 0..3 read the
-      // accumulator ----
-      if (cc_last) {
+      // ---- epilogue of the segment: warps 0..3 read the accumulator ----
+      if (seg_end) {
         if (warp < 4) {
-          const int db = tl & 1;
-          const uint32_t dph = static_cast<uint32_t>((tl >> 1) & 1);
+          const int db = sidx & 1;
+          const uint32_t dph = static_cast<uint32_t>((sidx >> 1) & 1);
           if (!dead && !mbar_wait(&dfull[db], dph)) dead = true;
           tc_fence_after();
           float d[16];
@@ -803,21 +848,67 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&dempty[db]);
-          const int row = tc * kMmaRows + 32 * warp + lane;
-          if (row < p.N) {
+          const int rt = 32 * warp + lane;  // row in the tile
+          const int row = tc * kMmaRows + rt;
+          if (whole_tile) {
+            if (row < p.N) {
+#pragma unroll
+              for (int m = 0; m < kMmaCols; ++m)
+                if (m < p.M) p.y[static_cast<size_t>(m) * p.N + row] = f32_to_bf16(d[m] * xinv[m]);
+            }
+          } else {
+            // a part of tile tc: leave it in this CTA's slot (0 for the
+            // range's first segment, 1 for its last), count it, and if it
+            // is the tile's last part to arrive, add all parts in CTA order
+            const long long ts = static_cast<long long>(tc) * p.nstage;
+            const int first = mma_range_of(ts, p.nsteps, gridDim.x);
+            const int last = mma_range_of(ts + p.nstage - 1, p.nsteps, gridDim.x);
+            float *mine = p.part + (static_cast<size_t>(blockIdx.x) * 2 + (v0 >= ts ? 0 : 1)) *
+                                       (kMmaCols * kMmaRows);
 #pragma unroll
             for (int m = 0; m < kMmaCols; ++m)
-              if (m < p.M) p.y[static_cast<size_t>(m) * p.N + row] = f32_to_bf16(d[m] * xinv[m]);
+              if (m < p.M) mine[m * kMmaRows + rt] = d[m];
+            __threadfence();
+            named_sync(2, 128);
+            if (warp == 0 && lane == 0)
+              *tile_flag = atomicAdd(&p.cnt[tc], 1) == last - first ? 1 : 0;
+            named_sync(2, 128);
+            if (*tile_flag) {
+              __threadfence();
+              float acc[16];
+#pragma unroll
+              for (int m = 0; m < kMmaCols; ++m) acc[m] = 0.f;
+              for (int j = first; j <= last; ++j) {
+                if (j == static_cast<int>(blockIdx.x)) {
+#pragma unroll
+                  for (int m = 0; m < kMmaCols; ++m) acc[m] += d[m];
+                } else {
+                  const long long sj = mma_range_start(j, p.nsteps, gridDim.x);
+                  const float *pj = p.part + (static_cast<size_t>(j) * 2 + (sj >= ts ? 0 : 1)) *
+                                                 (kMmaCols * kMmaRows);
+#pragma unroll
+                  for (int m = 0; m < kMmaCols; ++m)
+                    if (m < p.M) acc[m] += __ldcg(pj + m * kMmaRows + rt);
+                }
+              }
+              if (row < p.N) {
+#pragma unroll
+                for (int m = 0; m < kMmaCols; ++m)
+                  if (m < p.M)
+                    p.y[static_cast<size_t>(m) * p.N + row] = f32_to_bf16(acc[m] * xinv[m]);
+              }
+              if (warp == 0 && lane == 0) p.cnt[tc] = 0;  // ready for the next launch
+            }
           }
         }
-        ++tl;
+        ++sidx;
       }
     };
     Regs A, B;
-    if (t < p.ntiles) load(A, 0);
-    while (t < p.ntiles) {
+    if (v < v1) load(A, c);
+    while (v < v1) {
       step(A, B);
-      if (t >= p.ntiles) break;
+      if (v >= v1) break;
       step(B, A);
     }
     if (dead && p.err && lane == 0) atomicOr(p.err, 2);

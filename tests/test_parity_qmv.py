@@ -138,3 +138,17 @@ def test_qmv_batched_many_tiles_per_cta():
     rows = np.unique(np.concatenate([sample_rows(N, 300, seed=5), np.arange(N - 80, N)])).astype(np.int32)
     y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, rows=rows, nthreads=8)
     check(y[:, rows], y_ref, a_ref, "batched many tiles")
+
+
+def test_qmv_batched_split_tiles_repeatable():
+    # a few more 128-row tiles than SMs and four K stages per tile: the
+    # (tile, stage) steps are shared out evenly, so most tiles are cut into
+    # parts held by two CTAs and added by the last one to finish; the sum
+    # order is fixed, so repeated launches agree bit for bit, and the
+    # per-tile arrival counters start from zero again after each launch
+    M, N, K, bits, gs = 4, 150 * 128 - 20, 1024, 4, 32
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=8080)
+    ys = [run_qmv(x, w, s, b, M, N, K, bits, gs) for _ in range(3)]
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2])
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, nthreads=8)
+    check(ys[0], y_ref, a_ref, "batched split tiles")
