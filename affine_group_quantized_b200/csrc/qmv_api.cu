@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include <cuda_fp16.h>
 
@@ -36,6 +37,26 @@ int fail(int code, const char *fmt, ...) {
 int ok() {
   g_last_error.clear();
   return QMV_OK;
+}
+
+// Launch with programmatic stream serialization allowed: the kernel may be
+// scheduled while the previous kernel on the stream is finishing; it holds
+// its first global access until that kernel has completed (the kernels
+// start with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, int smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 bool aligned16(const void *p) {
@@ -256,7 +277,11 @@ int launch_t(const Plan &pl, cudaStream_t stream) {
                   cudaGetErrorString(e));
     granted = static_cast<int>(pl.smem);
   }
-  kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.p);
+  const cudaError_t le = launch_pdl(kern, pl.grid, pl.threads, pl.smem, stream, pl.p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(le));
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
@@ -414,7 +439,12 @@ int launch_mma_t(qmvk::MmaParams &mp, int grid, DeviceInfo *dev, cudaStream_t st
       return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     granted[d] = dev->smem_optin;
   }
-  kern<<<grid, qmvk::mma_threads<BITS>(), smem, stream>>>(tw, ts, tb, tx, mp);
+  const cudaError_t le =
+      launch_pdl(kern, grid, qmvk::mma_threads<BITS>(), smem, stream, tw, ts, tb, tx, mp);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(le));
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));

@@ -83,6 +83,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src,
       : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched right behind another on
+// the same stream may be scheduled before that one has finished; it waits
+// here, before its first global memory access, until the previous grid has
+// completed and its writes are visible (a no-op for an ordinary launch).
+// launch_dependents lets the next grid get scheduled as SMs free up.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // Named barrier `id` over `nthreads` threads (a multiple of 32): wait for
 // all of them, or only signal arrival without waiting.
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {

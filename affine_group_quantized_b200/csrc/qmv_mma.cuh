@@ -460,6 +460,8 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
   constexpr int nw = 4 * NP;  // dequant warps: 0 .. nw-1
   const int nst = p.nst;
   const uint32_t sbytes = p.stage_bytes;
+  grid_launch_dependents();
+  grid_dependency_wait();
 
   // ---- set-up: barriers, tensor memory, x row ranges ----
   if (warp == nw) {

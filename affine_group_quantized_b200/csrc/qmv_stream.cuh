@@ -733,6 +733,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t *empty = full + p.nslot;
   uint64_t *redfull = empty + p.nslot;
   uint64_t *redempty = redfull + p.nred;
+  grid_launch_dependents();
+  grid_dependency_wait();
 
   Groups g{};
   int nseg;
