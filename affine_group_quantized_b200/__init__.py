@@ -53,11 +53,12 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I = ctypes.c_void_p, ctypes.c_int
         L.qmv.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+        L.qmv_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
         L.qmv_gate_up.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.qmv_silu_gate_resid.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.gather_qmv.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
                                  P, P]
-        for f in (L.qmv, L.qmv_gate_up, L.qmv_silu_gate_resid, L.gather_qmv):
+        for f in (L.qmv, L.qmv_noalloc, L.qmv_gate_up, L.qmv_silu_gate_resid, L.gather_qmv):
             f.restype = I
         L.qmv_last_error.restype = ctypes.c_char_p
         L.qmv_last_error.argtypes = []
@@ -105,6 +106,13 @@ def qmv(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):
     """y[M,N] = x[M,K] @ dequant(w).T  (see include/qmv.h)."""
     _check("qmv", lib().qmv(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases),
                             _ptr(y), M, N, K, bits, group_size, _stream(stream)))
+
+
+def qmv_noalloc(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):
+    """qmv without device allocation by the library (see include/qmv.h)."""
+    _check("qmv_noalloc", lib().qmv_noalloc(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases),
+                                            _ptr(y), M, N, K, bits, group_size,
+                                            _stream(stream)))
 
 
 def qmv_gate_up(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up,

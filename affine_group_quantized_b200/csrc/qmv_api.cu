@@ -398,6 +398,40 @@ int mma_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
   return 0;
 }
 
+// The same scratch for qmv_noalloc, as a fixed array in the library's device
+// image: partial-sum slots for up to kStaticCtas CTAs, then arrival counters
+// for up to kStaticTiles tiles (zero at load; every launch leaves them zero).
+constexpr int kStaticCtas = 256;
+constexpr int kStaticTiles = 1 << 16;
+constexpr size_t kStaticPartBytes =
+    static_cast<size_t>(kStaticCtas) * 2 * qmvk::kMmaCols * qmvk::kMmaRows * 4;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticPartBytes +
+                                                                 kStaticTiles * 4];
+MmaScratch g_static_view[kMaxDevices];
+std::once_flag g_static_once[kMaxDevices];
+
+int static_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
+  if (sms > kStaticCtas || ntiles > kStaticTiles)
+    return fail(QMV_ERR_UNSUPPORTED,
+                "qmv_noalloc: %d SMs / %d row tiles exceed the fixed scratch (%d / %d)", sms,
+                ntiles, kStaticCtas, kStaticTiles);
+  cudaError_t e = cudaSuccess;
+  std::call_once(g_static_once[dev_id], [&] {
+    void *a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_static_scratch);
+    if (e == cudaSuccess) {
+      g_static_view[dev_id].part = static_cast<float *>(a);
+      g_static_view[dev_id].cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(a) +
+                                                          kStaticPartBytes);
+      g_static_view[dev_id].cnt_len = kStaticTiles;
+    }
+  });
+  if (!g_static_view[dev_id].part)
+    return fail(QMV_ERR_CUDA, "qmv_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+  *out = &g_static_view[dev_id];
+  return 0;
+}
+
 template <int BITS, int GS>
 int launch_mma_t(qmvk::MmaParams &mp, int grid, DeviceInfo *dev, cudaStream_t stream) {
   using ST = qmvk::MmaStage<BITS>;
@@ -463,7 +497,7 @@ int launch_mma_b(qmvk::MmaParams &mp, int gs, int grid, DeviceInfo *dev, cudaStr
 
 int launch_mma(const void *x, const uint32_t *w, const void *scales,
                const void *biases, void *y, int M, int N, int K, int bits, int gs,
-               DeviceInfo *dev, cudaStream_t stream) {
+               DeviceInfo *dev, cudaStream_t stream, bool fixed_scratch) {
   qmvk::MmaParams mp;
   std::memset(&mp, 0, sizeof mp);
   mp.w = reinterpret_cast<const uint8_t *>(w);
@@ -492,7 +526,9 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   cudaGetDevice(&d);
   MmaScratch *sc = nullptr;
   int rc;
-  if ((rc = mma_scratch(d, dev->sms, mp.ntiles, &sc))) return rc;
+  if ((rc = fixed_scratch ? static_scratch(d, dev->sms, mp.ntiles, &sc)
+                         : mma_scratch(d, dev->sms, mp.ntiles, &sc)))
+    return rc;
   mp.part = sc->part;
   mp.cnt = sc->cnt;
   switch (bits) {
@@ -503,30 +539,22 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   }
 }
 
-}  // namespace
-
-extern "C" {
-
-int qmv_abi_version(void) { return 1; }
-
-const char *qmv_last_error(void) { return g_last_error.c_str(); }
-
-int qmv(const void *x, const uint32_t *w, const void *scales,
-        const void *biases, void *y, int M, int N, int K, int bits,
-        int group_size, void *stream) {
+int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *scales,
+             const void *biases, void *y, int M, int N, int K, int bits, int group_size,
+             void *stream, bool fixed_scratch) {
   if (!x || !w || !scales || !biases || !y)
-    return fail(QMV_ERR_NULL, "qmv: a buffer pointer is NULL");
+    return fail(QMV_ERR_NULL, "%s: a buffer pointer is NULL", name);
   int rc = check_common(N, K, bits, group_size);
   if (rc) return rc;
-  if (M <= 0) return fail(QMV_ERR_SHAPE, "qmv: M=%d must be positive", M);
+  if (M <= 0) return fail(QMV_ERR_SHAPE, "%s: M=%d must be positive", name, M);
   if (!aligned16(x) || !aligned16(w) || !aligned16(scales) ||
       !aligned16(biases) || !aligned16(y))
-    return fail(QMV_ERR_ALIGN, "qmv: buffers must be 16-byte aligned");
+    return fail(QMV_ERR_ALIGN, "%s: buffers must be 16-byte aligned", name);
   DeviceInfo *dev;
   if ((rc = device_info(&dev))) return rc;
   if (mma_path(M, K, bits, group_size))
     return launch_mma(x, w, scales, biases, y, M, N, K, bits, group_size, dev,
-                      static_cast<cudaStream_t>(stream));
+                      static_cast<cudaStream_t>(stream), fixed_scratch);
   Plan pl;
   init_params(pl.p);
   qmvk::StreamParams &p = pl.p;
@@ -543,6 +571,26 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
   p.total_rows = N;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int qmv_abi_version(void) { return 1; }
+
+const char *qmv_last_error(void) { return g_last_error.c_str(); }
+
+int qmv(const void *x, const uint32_t *w, const void *scales,
+        const void *biases, void *y, int M, int N, int K, int bits,
+        int group_size, void *stream) {
+  return qmv_impl("qmv", x, w, scales, biases, y, M, N, K, bits, group_size, stream, false);
+}
+
+int qmv_noalloc(const void *x, const uint32_t *w, const void *scales, const void *biases,
+                void *y, int M, int N, int K, int bits, int group_size, void *stream) {
+  return qmv_impl("qmv_noalloc", x, w, scales, biases, y, M, N, K, bits, group_size, stream,
+                  true);
 }
 
 int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,

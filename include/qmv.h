@@ -80,6 +80,22 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
         int group_size, void *stream);
 
 /*
+ * qmv_noalloc -- the same operation, arguments and layouts as qmv, with no
+ * device memory allocated by the library.  qmv's tensor-core path (several
+ * activation rows, 2/4/8-bit codes) adds up 128-row tiles that are split
+ * between CTAs through scratch memory the library allocates on first use;
+ * qmv_noalloc takes that scratch from a fixed array in the library's device
+ * image instead (its address from cudaGetSymbolAddress, per device).
+ * Results are identical to qmv's for the same inputs.
+ *   returns QMV_ERR_UNSUPPORTED when the call would need more than the array
+ *   holds: more than 256 SMs, or more than 65536 row tiles (N > 8388608).
+ * Calls on one device that use the array are expected in stream order.
+ */
+int qmv_noalloc(const void *x, const uint32_t *w, const void *scales,
+                const void *biases, void *y, int M, int N, int K, int bits,
+                int group_size, void *stream);
+
+/*
  * qmv_gate_up -- dual-output GEMV over one input, in ONE kernel launch:
  *   y_gate = x @ dequant(W_gate).T,   y_up = x @ dequant(W_up).T
  *
