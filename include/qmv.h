@@ -74,6 +74,14 @@ typedef enum {
  *   biases  bf16 [N, K/group_size]
  *   y       bf16 [M, N]  (written; must not overlap the inputs)
  *   y[m][n] = sum_k x[m][k] * w_hat[n][k]
+ *
+ * M = 3 .. 16 with 2-, 4- or 8-bit codes (K a multiple of 1024/bits,
+ * K/group_size a multiple of 8) runs on the tensor cores: each w_hat is
+ * rounded once to fp16 and each x row is scaled by a power of two into fp16
+ * range, with fp32 accumulation; scales and biases should lie in fp16's
+ * normal range (magnitude 2^-14 .. 65504) there.  The first such call on a
+ * device allocates the path's scratch (2.4 MB plus 4 bytes per 128 rows);
+ * qmv_noalloc does the same without allocating.
  */
 int qmv(const void *x, const uint32_t *w, const void *scales,
         const void *biases, void *y, int M, int N, int K, int bits,
