@@ -405,14 +405,24 @@ __device__ __noinline__ void plain_tail(uint32_t dst, const uint8_t *src,
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
+// The weights, scales and biases are read once per launch: their lines are
+// marked first to go in L2, so the stream does not push out what is reused
+// (the kernel's own code, activations, outputs).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const uint8_t *src,
                                           uint32_t bytes, uint64_t *bar) {
+  const uint64_t pol = l2_evict_first_policy();
   for (uint32_t o = 0; o < bytes; o += kBulkChunk) {
     const uint32_t n = bytes - o < kBulkChunk ? bytes - o : kBulkChunk;
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1], %2, [%3];\n" ::"r"(dst + o),
-        "l"(src + o), "r"(n), "r"(smem_u32(bar))
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;\n" ::"r"(dst + o),
+        "l"(src + o), "r"(n), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
   }
 }
@@ -433,6 +443,7 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
   SlotPos pos{0, 0u};
   long long nslots = 0;  // slots filled so far
   bool failed = false;
+  bool waited = false;
   while (tw.next(t)) {
     const int ns_t = tile_slots(p, t.nrows);
     const bool active = q < ns_t;
@@ -447,6 +458,10 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
     }
     uint32_t dw = 0, ds = 0, bw = 0, bs = 0;
     const uint8_t *wsrc = nullptr, *ssrc = nullptr, *bsrc = nullptr;
+    if (!waited) {
+      grid_dependency_wait();
+      waited = true;
+    }
     if (active) {
       const Seg sg = seg_info<MR>(p, g, t.seg);
       const int w_arr = p.mode == MODE_GATHER ? 0 : sg.arr;
@@ -501,6 +516,7 @@ __device__ __forceinline__ void epilogue_loop(const StreamParams &p,
                                               uint64_t *redempty,
                                               const Groups &g, int nseg,
                                               int lane) {
+  grid_dependency_wait();
   TileWalker tw;
   tw.init(nseg, p.N, p.RT, p.tps, p.nred, p.mode == MODE_GATHER);
   Tile t;
@@ -734,11 +750,14 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t *redfull = empty + p.nslot;
   uint64_t *redempty = redfull + p.nred;
   grid_launch_dependents();
-  grid_dependency_wait();
+  // Each role waits for the previous grid just before its first global
+  // access, so that its set-up code runs (and is fetched) while that grid
+  // drains; the gather mode reads its index arrays first.
 
   Groups g{};
   int nseg;
   if (p.mode == MODE_GATHER) {
+    grid_dependency_wait();
     g = groups_at(smem, p);
     build_groups<MR>(p, g, tid, blockDim.x);  // ends with __syncthreads
     nseg = *g.nseg;
@@ -801,6 +820,7 @@ __global__ void __launch_bounds__(512, 1)
   // producer sets up and starts the weight stream, so that these few lines
   // are not queued behind it in HBM.  The mbarriers are used only after
   // named barrier 1, which the producer passes once it has set them up.
+  grid_dependency_wait();
   {
     TileWalker w0 = tw;
     Tile t0;

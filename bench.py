@@ -293,7 +293,11 @@ def run_ours(args):
     # events, which then give the value).
     flush = step_bytes < 64 * 2**20
     copies = 1 if flush else max(2, -(-2 * L2_BYTES // step_bytes) + 1)
-    dls = [DeviceLaunch(l, copies, torch) for l in launches]
+    # Each launch also gets enough weight copies that timing it alone (below)
+    # streams more than twice the L2 capacity between two reads of the same
+    # bytes; a step uses the first `copies` of them.
+    dls = [DeviceLaunch(l, copies if flush else max(copies, -(-2 * L2_BYTES // l.nbytes) + 1),
+                        torch) for l in launches]
     scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if flush else None
 
     def step(k):
@@ -348,11 +352,12 @@ def run_ours(args):
         ms = float(tt.item())
 
     # Average duration of each launch: a graph of R back-to-back launches of
-    # that kernel alone (rotating weight copies; L2 scrubbed first for the
-    # small workloads), timed with events around the replays.
+    # that kernel alone (rotating through all of its weight copies, more than
+    # twice the L2 capacity; L2 scrubbed first for the small workloads), timed
+    # with events around the replays.
     dur = []
     for dl in dls:
-        R = 3 * copies
+        R = 3 * len(dl.copies)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for r in range(R):
@@ -443,7 +448,9 @@ def run_ours(args):
         "config": dict(cfg, l2=(f"L2 flushed before every step ({2 * L2_BYTES >> 20} MiB "
                                 f"write); value from per-launch events" if flush else
                                 f"inputs larger than L2: {copies} rotating weight copies, "
-                                f"{step_bytes * copies / 2**20:.0f} MiB between reuse"),
+                                f"{step_bytes * copies / 2**20:.0f} MiB between reuse; each "
+                                f"launch timed alone rotates through more than "
+                                f"{2 * L2_BYTES >> 20} MiB of its own copies"),
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        graphs=f"timed steps replayed as CUDA graphs of {copies} steps (one "
                               f"weight rotation); the remainder one step per graph"),
