@@ -248,14 +248,26 @@ __device__ __forceinline__ uint32_t lds16_mma(uint32_t a) {
   return v;
 }
 // 2-D tensor copy global -> shared (box of the tensor map at (x, y)),
-// completing its bytes on `bar`.
+// completing its bytes on `bar`, with an L2 cache policy (the weights,
+// scales and biases are read once per launch: evict-first, so they do not
+// push the kernel's code and the activations out of L2).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
+                                            uint64_t *bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
 }
 
 // NG consecutive bf16 values (NG = 1, 2, 4, 8; aligned to NG) from shared
@@ -461,7 +473,6 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
   const int nst = p.nst;
   const uint32_t sbytes = p.stage_bytes;
   grid_launch_dependents();
-  grid_dependency_wait();
 
   // ---- set-up: barriers, tensor memory, x row ranges ----
   if (warp == nw) {
@@ -487,6 +498,9 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
+  // the first global access of every thread follows (x, then the copies and
+  // the stores): wait for the previous grid here, after the on-chip set-up
+  grid_dependency_wait();
   __syncthreads();
   if (warp < nw) {
     // max |x| of each x row, over all K, by all dequant threads
@@ -553,6 +567,8 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
       bool dead = false;
       constexpr int XS = mma_x_slice<BITS>();
       const uint32_t tx = ST::tx_bytes(p.M);
+      const uint64_t pol_stream = l2_policy_evict_first();  // read once
+      const uint64_t pol_keep = l2_policy_evict_last();     // x: read by every tile
       const uint32_t xstep = p.M * ST::x_row;
       int t = static_cast<int>(v0 / p.nstage), c = static_cast<int>(v0 % p.nstage);
       for (long long v = v0; v < v1; ++v, ++issued) {
@@ -563,13 +579,14 @@ __global__ void __launch_bounds__(mma_threads<BITS>(), 1)
           const uint32_t dst = ring + sp.idx * sbytes;
           uint64_t *bar = &wfull[sp.idx];
           mbar_arrive_expect_tx(bar, tx);
-          tma_load_2d(dst, &tm_w, c * 128, r0, bar);
+          tma_load_2d(dst, &tm_w, c * 128, r0, bar, pol_stream);
           const int wg = (c * (SC / GS)) & ~7;
-          tma_load_2d(dst + ST::s_off, &tm_s, wg, r0, bar);
-          tma_load_2d(dst + ST::b_off, &tm_b, wg, r0, bar);
+          tma_load_2d(dst + ST::s_off, &tm_s, wg, r0, bar, pol_stream);
+          tma_load_2d(dst + ST::b_off, &tm_b, wg, r0, bar, pol_stream);
 #pragma unroll
           for (int xs = 0; xs < SC / XS; ++xs)
-            tma_load_2d(dst + ST::x_off + xs * xstep, &tm_x, c * SC + xs * XS, 0, bar);
+            tma_load_2d(dst + ST::x_off + xs * xstep, &tm_x, c * SC + xs * XS, 0, bar,
+                        pol_keep);
           sp.next(nst);
         }
         if (++c == p.nstage) {
