@@ -144,8 +144,8 @@ struct Plan {
 // Rows per consumer thread per tile; the same rule as the kernel's
 // rows_per_thread<BITS, MR, NSL>().
 int rows_per_thread_host(int bits, int mr, int nsl) {
-  const int base = (bits == 2 || bits == 3 || bits == 4) ? 16 : 8;
-  return (mr * nsl == 1) ? base : base / 2;
+  (void)bits;
+  return (mr * nsl == 1) ? 8 : 4;
 }
 
 // Thread layout: Upad (>= 32, a multiple of 32) consumer threads cover the
@@ -174,13 +174,13 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   const int ra_s = 16 / gcd_i((2 * G) % 16 == 0 ? 16 : (2 * G) % 16, 16);
   const int RA = ra_w * ra_s / gcd_i(ra_w, ra_s);
   const int wpr = Upad / 32 / nsl;
-  // consumer threads: up to 448 (plus producer and epilogue warps: 512 per
-  // CTA, 128 registers per thread).  A slot holds SR rows of every row
+  // consumer threads: up to 512 (plus producer and epilogue warps: 576 per
+  // CTA, at most 113 registers per thread).  A slot holds SR rows of every row
   // phase (SR = 2 * pairs per slot, the kernel's pairs_per_slot<BITS>); the
   // ring must hold the slots of two tiles (RPT / SR each), so the row phases
   // are reduced until it does.
   const int SR = 2 * 2;  // the kernel's 2 * pairs_per_slot<BITS>()
-  const int tc_max = 448;
+  const int tc_max = 512;
   int PH = nsl == 1 && Upad <= tc_max ? tc_max / Upad : 1;
   struct Sizes { long long w, s, red, slot; };
   auto sizes = [&](int ph) {

@@ -687,12 +687,12 @@ __host__ __device__ constexpr int pairs_per_slot() {
   return 2;
 }
 
-// Rows per consumer thread per tile (a compile-time constant per code width):
-// the rows handed to the epilogue at once.
+// Rows per consumer thread per tile: the rows handed to the epilogue at once.
+// Eight (four with two units or two activation rows per thread) keeps two
+// tiles of the ring within shared memory with up to 16 consumer warps.
 template <int BITS, int MR, int NSL>
 __host__ __device__ constexpr int rows_per_thread() {
-  constexpr int base = (BITS == 2 || BITS == 3 || BITS == 4) ? 16 : 8;
-  return (MR * NSL == 1) ? base : base / 2;
+  return (MR * NSL == 1) ? 8 : 4;
 }
 
 // Partial sums of two rows of the thread's unit: decode, dot products, group
@@ -737,7 +737,7 @@ __device__ __forceinline__ void row_pair_dot(const uint32_t (&w0)[BITS],
 // consumer thread (1 or 2); SILU: the activations are silu(gate) * up
 // (MODE_SILU only, a separate kernel so the others carry none of its code).
 template <int BITS, int MR, int NSL, bool SILU>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(576, 1)
     qmv_stream_kernel(const StreamParams p) {
   constexpr int RPT = rows_per_thread<BITS, MR, NSL>();
   extern __shared__ __align__(128) unsigned char smem[];
