@@ -136,6 +136,7 @@ int check_common(int N, int K, int bits, int gs) {
 struct Plan {
   qmvk::StreamParams p;
   int mr = 1, nsl = 1;
+  bool big = false;  // taller tiles (gather mode)
   int threads = 0;
   size_t smem = 0;
   int grid = 0;
@@ -143,9 +144,9 @@ struct Plan {
 
 // Rows per consumer thread per tile; the same rule as the kernel's
 // rows_per_thread<BITS, MR, NSL>().
-int rows_per_thread_host(int bits, int mr, int nsl) {
-  (void)bits;
-  return (mr * nsl == 1) ? 8 : 4;
+int rows_per_thread_host(int bits, int mr, int nsl, bool big) {
+  const int base = big && (bits == 2 || bits == 3 || bits == 4) ? 16 : 8;
+  return (mr * nsl == 1) ? base : base / 2;
 }
 
 // Thread layout: Upad (>= 32, a multiple of 32) consumer threads cover the
@@ -166,7 +167,8 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   const int mr = (nsl == 1 && mr_want >= 2) ? 2 : 1;
   const long long row_bytes = static_cast<long long>(K) * bits / 8;
   const int G = K / gs;
-  const int RPT = rows_per_thread_host(bits, mr, nsl);
+  const bool big = p.mode == qmvk::MODE_GATHER;
+  const int RPT = rows_per_thread_host(bits, mr, nsl, big);
   long long grp_bytes = 0;
   if (p.mode == qmvk::MODE_GATHER)
     grp_bytes = (2LL * p.num_experts + 3LL * p.num_pairs + 1) * 4;
@@ -180,7 +182,7 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   // ring must hold the slots of two tiles (RPT / SR each), so the row phases
   // are reduced until it does.
   const int SR = 2 * 2;  // the kernel's 2 * pairs_per_slot<BITS>()
-  const int tc_max = 512;
+  const int tc_max = big ? 448 : 512;
   int PH = nsl == 1 && Upad <= tc_max ? tc_max / Upad : 1;
   struct Sizes { long long w, s, red, slot; };
   auto sizes = [&](int ph) {
@@ -221,6 +223,7 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   p.wpr = wpr;
   p.row_bytes = static_cast<uint32_t>(row_bytes);
   p.nch = p.mode == qmvk::MODE_GATHER ? 1 : (p.M + mr - 1) / mr;
+  p.read_once = p.mode != qmvk::MODE_GATHER && p.nch == 1;
   p.w_slot = static_cast<uint32_t>(z.w);
   p.s_slot = static_cast<uint32_t>(z.s);
   const long long ring = ns * z.slot;
@@ -231,6 +234,7 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   pl.smem = static_cast<size_t>(p.grp_off + grp_bytes);
   pl.mr = mr;
   pl.nsl = nsl;
+  pl.big = big;
   pl.threads = Tc + 64;
   // One CTA per SM (fewer when there are fewer tiles).  Tiles are dealt
   // round-robin, so the tile height is lowered until every CTA gets the
@@ -256,18 +260,18 @@ int make_plan(Plan &pl, int bits, int gs, int mr_want, DeviceInfo *dev) {
   return QMV_OK;
 }
 
-template <int BITS, int MR, int NSL, bool SILU>
+template <int BITS, int MR, int NSL, bool SILU, bool BIG>
 int &granted_smem(int dev) {
   static int granted[kMaxDevices] = {};
   return granted[dev];
 }
 
-template <int BITS, int MR, int NSL, bool SILU>
+template <int BITS, int MR, int NSL, bool SILU, bool BIG = false>
 int launch_t(const Plan &pl, cudaStream_t stream) {
-  auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL, SILU>;
+  auto kern = qmvk::qmv_stream_kernel<BITS, MR, NSL, SILU, BIG>;
   int dev = 0;
   cudaGetDevice(&dev);
-  int &granted = granted_smem<BITS, MR, NSL, SILU>(dev);
+  int &granted = granted_smem<BITS, MR, NSL, SILU, BIG>(dev);
   if (static_cast<int>(pl.smem) > granted) {
     cudaError_t e = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -290,6 +294,13 @@ int launch_t(const Plan &pl, cudaStream_t stream) {
 
 template <int BITS, bool SILU>
 int launch_shape(const Plan &pl, cudaStream_t stream) {
+  if constexpr (!SILU) {
+    if (pl.big) {  // gather mode: taller tiles
+      if (pl.nsl == 2) return launch_t<BITS, 1, 2, false, true>(pl, stream);
+      if (pl.mr == 2) return launch_t<BITS, 2, 1, false, true>(pl, stream);
+      return launch_t<BITS, 1, 1, false, true>(pl, stream);
+    }
+  }
   if (pl.nsl == 2) return launch_t<BITS, 1, 2, SILU>(pl, stream);
   if (pl.mr == 2) return launch_t<BITS, 2, 1, SILU>(pl, stream);
   return launch_t<BITS, 1, 1, SILU>(pl, stream);

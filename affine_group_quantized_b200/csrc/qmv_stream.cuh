@@ -63,6 +63,7 @@ struct StreamParams {
   int tps;                // tiles per segment: ceil(N / RT)
   int full_slots;         // slots of a full tile: ceil(RT / slot_rows)
   int RA;                 // row alignment making copy starts 16-byte aligned
+  int read_once;          // every weight row is streamed once per launch
   int nmat;               // weight matrices (1, or 2 for gate/up)
   int nch;                // activation chunks per matrix: ceil(M / MR)
   int nslot;              // slots in the shared-memory weight ring
@@ -405,18 +406,22 @@ __device__ __noinline__ void plain_tail(uint32_t dst, const uint8_t *src,
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
-// The weights, scales and biases are read once per launch: their lines are
-// marked first to go in L2, so the stream does not push out what is reused
-// (the kernel's own code, activations, outputs).
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+// When every weight row is streamed once per launch, the weights, scales
+// and biases are marked first to go in L2, so the stream does not push out
+// what is reused (the kernel's own code, activations, outputs).  Rows read
+// again (several chunks of activation rows, or experts revisited by the
+// gather mode) keep the normal policy.
+__device__ __forceinline__ uint64_t l2_stream_policy(bool read_once) {
   uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  if (read_once)
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;\n" : "=l"(pol));
   return pol;
 }
 
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const uint8_t *src,
-                                          uint32_t bytes, uint64_t *bar) {
-  const uint64_t pol = l2_evict_first_policy();
+                                          uint32_t bytes, uint64_t *bar, uint64_t pol) {
   for (uint32_t o = 0; o < bytes; o += kBulkChunk) {
     const uint32_t n = bytes - o < kBulkChunk ? bytes - o : kBulkChunk;
     asm volatile(
@@ -487,9 +492,10 @@ __device__ __forceinline__ void producer_loop(const StreamParams &p,
     if (active) {
       uint64_t *bar = &full[my.idx];
       mbar_arrive_expect_tx(bar, bw + 2 * bs);
-      bulk_copy(dw, wsrc, bw, bar);
-      bulk_copy(ds, ssrc, bs, bar);
-      bulk_copy(ds + p.s_slot, bsrc, bs, bar);
+      const uint64_t pol = l2_stream_policy(p.read_once != 0);
+      bulk_copy(dw, wsrc, bw, bar, pol);
+      bulk_copy(ds, ssrc, bs, bar, pol);
+      bulk_copy(ds + p.s_slot, bsrc, bs, bar, pol);
     }
     pos = pos.plus(ns_t, p.nslot);
     nslots += ns_t;
@@ -689,10 +695,14 @@ __host__ __device__ constexpr int pairs_per_slot() {
 
 // Rows per consumer thread per tile: the rows handed to the epilogue at once.
 // Eight (four with two units or two activation rows per thread) keeps two
-// tiles of the ring within shared memory with up to 16 consumer warps.
-template <int BITS, int MR, int NSL>
+// tiles of the ring within shared memory with up to 16 consumer warps.  The
+// gather mode (BIG) keeps taller tiles, 16 rows for codes of up to 4 bits,
+// with at most 14 consumer warps: its expert segments are short, and each
+// tile pays a reduction and, at a segment change, an activation reload.
+template <int BITS, int MR, int NSL, bool BIG = false>
 __host__ __device__ constexpr int rows_per_thread() {
-  return (MR * NSL == 1) ? 8 : 4;
+  constexpr int base = BIG && (BITS == 2 || BITS == 3 || BITS == 4) ? 16 : 8;
+  return (MR * NSL == 1) ? base : base / 2;
 }
 
 // Partial sums of two rows of the thread's unit: decode, dot products, group
@@ -736,10 +746,10 @@ __device__ __forceinline__ void row_pair_dot(const uint32_t (&w0)[BITS],
 // BITS: code width; MR: activation rows per segment (1 or 2); NSL: units per
 // consumer thread (1 or 2); SILU: the activations are silu(gate) * up
 // (MODE_SILU only, a separate kernel so the others carry none of its code).
-template <int BITS, int MR, int NSL, bool SILU>
-__global__ void __launch_bounds__(576, 1)
+template <int BITS, int MR, int NSL, bool SILU, bool BIG = false>
+__global__ void __launch_bounds__(BIG ? 512 : 576, 1)
     qmv_stream_kernel(const StreamParams p) {
-  constexpr int RPT = rows_per_thread<BITS, MR, NSL>();
+  constexpr int RPT = rows_per_thread<BITS, MR, NSL, BIG>();
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
   const int Tc = p.Upad * p.PH / NSL;  // consumer threads
