@@ -143,7 +143,7 @@ struct Plan {
 };
 
 // Rows per consumer thread per tile; the same rule as the kernel's
-// rows_per_thread<BITS, MR, NSL>().
+// rows_per_thread<BITS, MR, NSL, BIG>() (BIG: the gather mode).
 int rows_per_thread_host(int bits, int mr, int nsl, bool big) {
   const int base = big && (bits == 2 || bits == 3 || bits == 4) ? 16 : 8;
   return (mr * nsl == 1) ? base : base / 2;

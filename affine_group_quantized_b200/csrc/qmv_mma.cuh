@@ -12,23 +12,26 @@
 //     rows (128-byte swizzle), the matching window of each row's scales and
 //     of its biases (32-byte swizzle), and the stage's slice of the M live x
 //     rows; rows past N arrive as zeros;
-//   * dequant warps (16): turn each stage into fp16 weights
-//     w_hat = scale * q + bias (codes made exact fp16 values with the
-//     0x6400 magic, then one half2 FMA: a single rounding, relative error
-//     below 2^-11) and write them straight into tensor memory, where the MMA
-//     takes its A operand (row r of the tile is tensor-memory lane r, so
-//     each warp writes the rows of its own lane quarter); the chunk of x
-//     becomes the fp16 B operand in shared memory (each x row scaled by its
-//     own power of two into fp16 range, undone in the epilogue); after a
-//     tile's last chunk they read the accumulator and store y;
+//   * dequant warps (8; 16 for 2-bit codes): turn each stage into fp16
+//     weights w_hat = scale * q + bias (a code made an exact fp16 value with
+//     the 0x6400 magic, an exact fp16 correction, then one half2 FMA: a
+//     single rounding, relative error below 2^-11) and write them straight
+//     into tensor memory, where the MMA takes its A operand (row r of the
+//     tile is tensor-memory lane r, so each warp writes the rows of its own
+//     lane quarter); the chunk of x becomes the fp16 B operand in shared
+//     memory (each x row scaled by its own power of two into fp16 range,
+//     undone in the epilogue); at the end of a segment (the CTA's steps in
+//     one tile) warps 0-3 read the accumulators and store y, or leave a
+//     partial sum for the CTA that completes the tile;
 //   * MMA warp: one thread issues the chunk's eight MMAs and commits them
 //     to mbarriers; the warp also owns the tensor-memory allocation.
 // Keeping A out of shared memory matters: in fp16 the weights are 4x (4-bit)
 // to 8x (2-bit) their packed size, and writing them to shared memory and
 // reading them back through the tensor core's descriptor path would cost
 // more shared-memory bandwidth than the HBM stream delivers.
-// The accumulator is double-buffered in tensor memory (two 16-column
-// halves), so one tile's epilogue overlaps the next tile's MMAs.
+// The accumulators are double-buffered in tensor memory (two sets of
+// kMmaNacc 16-column accumulators), so one segment's epilogue overlaps the
+// next segment's MMAs.
 //
 // The order of k inside each group of 8 is permuted identically in W_hat
 // and X^T (the nibble / byte pairing of the half2 unpack); a contraction
