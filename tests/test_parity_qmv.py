@@ -74,6 +74,27 @@ def test_qmv_negative_scales_and_extreme_activations():
     check(y, y_ref, a_ref, "negative scales / extreme x")
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+def test_qmv_batched_negative_scales_and_extreme_activations(bits):
+    # the tensor-core path (four activation rows): sign-flipped scales, a
+    # huge and a tiny unit in one row (the row's power-of-two fp16 range is
+    # set by its largest value), exact zeros and an all-zero unit
+    gs, M, N, K = 32, 4, 300, 1024
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=17 + bits)
+    s = s ^ np.where(np.arange(s.size).reshape(s.shape) % 3 == 0,
+                     np.uint16(0x8000), np.uint16(0))
+    xf = synth.bits_to_float(x).astype(np.float32).copy()
+    xf[0, :256] *= np.float32(2.0 ** 60)
+    xf[0, 256:512] *= np.float32(2.0 ** -60)
+    xf[1, 100] = 0.0
+    xf[2, 512:544] = 0.0
+    xf[3, :] *= np.float32(2.0 ** -100)   # a whole row far below 1
+    x = synth.bf16_bits(torch.from_numpy(xf))
+    y = run_qmv(x, w, s, b, M, N, K, bits, gs)
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs)
+    check(y, y_ref, a_ref, f"batched negative scales / extreme x bits={bits}")
+
+
 @pytest.mark.parametrize("gs", [32, 128])
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
 def test_qmv_batched_full_size(M, gs):

@@ -15,6 +15,29 @@ def test_noalloc_is_exported_and_bound():
     assert callable(agq.qmv_noalloc)
 
 
+A = 0x10000  # a 16-byte aligned fake device address; never dereferenced
+
+
+def test_noalloc_argument_checks():
+    # the same host-side checks as qmv, before any device is touched
+    f = agq.lib().qmv_noalloc
+    ok_args = [A, A, A, A, A, 4, 64, 1024, 4, 64, None]
+    names = ["x", "w", "s", "b", "y", "M", "N", "K", "bits", "gs", "stream"]
+
+    def call(**over):
+        a = list(ok_args)
+        for k, v in over.items():
+            a[names.index(k)] = v
+        return f(*a)
+
+    assert call(w=None) == agq.QMV_ERR_NULL
+    assert "qmv_noalloc" in agq.last_error()
+    assert call(bits=7) == agq.QMV_ERR_UNSUPPORTED
+    assert call(K=96) == agq.QMV_ERR_SHAPE
+    assert call(M=0) == agq.QMV_ERR_SHAPE
+    assert call(y=A + 8) == agq.QMV_ERR_ALIGN
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("M, N, K, bits, gs", [
     (4, 150 * 128 - 20, 1024, 4, 32),  # tensor cores, tiles split between CTAs
