@@ -270,6 +270,23 @@ def recorded_traffic(kernel_label, workload_name):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(value, device):
+    """The largest of `value` over the ranks of the default process group
+    (the slowest replica times the job); the value itself with one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_step, steps, ms):
+    """Whole-job throughput: every replica's bytes over the slowest time."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -345,11 +362,7 @@ def run_ours(args):
             graphs[k].replay()
         t1.record(stream)
         torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
 
     # Average duration of each launch: a graph of R back-to-back launches of
     # that kernel alone (rotating through all of its weight copies, more than
@@ -421,11 +434,7 @@ def run_ours(args):
         egraphs[k % copies].replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
     del graphs, egraphs
 
     peak, peak_kind = measured_peaks()
@@ -437,7 +446,7 @@ def run_ours(args):
                         "bytes": l.nbytes}
     dom = max(range(len(dls)), key=lambda i: dur[i])
     ach = launches[dom].nbytes / (dur[dom] * 1e-3) / 1e9
-    value = world * step_bytes * K / (ms * 1e-3) / 1e9
+    value = job_gbs(world, step_bytes, K, ms)
     if flush:  # the step region includes the L2 scrub: use kernel time only
         value = world * step_bytes / (sum(dur) * 1e-3) / 1e9
     out = {
@@ -462,7 +471,7 @@ def run_ours(args):
         "per_launch": per,
         "tokens_per_s_equiv": {l.label: round(1e6 / (d * 1e3), 1)
                                for l, d in zip(launches, dur)},
-        "e2e": {"value": round(world * step_bytes * K / (e2e_ms * 1e-3) / 1e9, 1),
+        "e2e": {"value": round(job_gbs(world, step_bytes, K, e2e_ms), 1),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "weights resident in HBM (decode); x copied in and y copied "
                         "out every step; each step replayed as one CUDA graph"},
