@@ -1,0 +1,170 @@
+"""Host-side logic of bench.py, checked on the CPU: the algorithmic byte
+counts behind every GB/s figure, the clock sampler's decoding of NVML's
+clock-event reasons (against a fake NVML), and the lookups of the measured
+peak and of the recorded DRAM traffic."""
+import json
+import os
+import sys
+import time
+import types
+
+import numpy as np
+import pytest
+
+import bench
+
+
+def _arrays_bytes(*arrays):
+    return sum(np.asarray(a).nbytes for a in arrays)
+
+
+@pytest.mark.parametrize("name", ["qmv_small", "decode_sweep"])
+def test_qmv_bytes_are_the_arrays_read_and_written(name):
+    # read: packed codes, scales, biases, activations; written: bf16 y
+    launches, _ = bench.workload(name)
+    for l in launches:
+        assert l.nbytes == _arrays_bytes(l.w, l.s, l.b, l.x) + 2 * l.M * l.N, l.label
+
+
+def test_ffn_bytes_are_the_arrays_read_and_written():
+    gate_up, silu = bench.workload("ffn_int8")[0]
+    # gate/up: two weight sets, one x; two bf16 outputs of N
+    assert gate_up.nbytes == (_arrays_bytes(gate_up.wg, gate_up.sg, gate_up.bg,
+                                            gate_up.wu, gate_up.su, gate_up.bu,
+                                            gate_up.x) + 2 * 2 * gate_up.N)
+    # SiLU down: its weights and residual, the gate and up vectors (bf16 of
+    # its K) and the bf16 output of its N
+    assert silu.nbytes == (_arrays_bytes(silu.w, silu.s, silu.b, silu.resid) +
+                           2 * 2 * silu.K + 2 * silu.N)
+
+
+def test_gather_bytes_count_touched_experts_only():
+    launches, cfg = bench.workload("moe_gather")
+    for l in launches:
+        touched = np.unique(l.rhs)
+        assert len(touched) == cfg["touched_experts"]
+        per_w = l.w.nbytes // l.E
+        per_sb = l.s.nbytes // l.E
+        weights = len(touched) * (per_w + 2 * per_sb)
+        index = _arrays_bytes(l.lhs, l.rhs)
+        assert l.nbytes == weights + l.x.nbytes + 2 * l.P * l.N + index, l.label
+
+
+class _FakeNvml(types.ModuleType):
+    """NVML stand-in: fixed clock readings and event-reason masks."""
+
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, masks, fail_init=False):
+        super().__init__("pynvml")
+        self._clocks, self._masks, self._fail = list(clocks), list(masks), fail_init
+        self.calls = 0
+
+    def nvmlInit(self):
+        if self._fail:
+            raise RuntimeError("NVML Shared Library Not Found")
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        assert uuid.startswith("GPU-")
+        return "handle"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, clock):
+        assert h == "handle" and clock == self.NVML_CLOCK_SM
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, clock):
+        i = min(self.calls, len(self._clocks) - 1)
+        self.calls += 1
+        return self._clocks[i]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self._masks[min(self.calls - 1, len(self._masks) - 1)]
+
+
+def _fake_torch():
+    props = types.SimpleNamespace(uuid="0d4e5c6a-0000-0000-0000-000000000001")
+    cuda = types.SimpleNamespace(current_device=lambda: 0,
+                                 get_device_properties=lambda i: props)
+    return types.SimpleNamespace(cuda=cuda)
+
+
+def test_clock_reason_bits_are_nvml_constants():
+    nv = pytest.importorskip("pynvml")
+    names = {"gpu_idle": "GpuIdle", "applications_clocks_setting": "ApplicationsClocksSetting",
+             "sw_power_cap": "SwPowerCap", "hw_slowdown": "HwSlowdown",
+             "sync_boost": "SyncBoost", "sw_thermal_slowdown": "SwThermalSlowdown",
+             "hw_thermal_slowdown": "HwThermalSlowdown",
+             "hw_power_brake_slowdown": "HwPowerBrakeSlowdown",
+             "display_clock_setting": "DisplayClockSetting"}
+    for bit, name in bench.ClockSampler._REASONS.items():
+        assert getattr(nv, "nvmlClocksEventReason" + names[name]) == bit, name
+
+
+def test_clock_sampler_decodes_reasons_and_takes_the_median(monkeypatch):
+    fake = _FakeNvml(clocks=[1965, 1950, 1965, 1300, 1965],
+                     masks=[0x1, 0x4, 0x4 | 0x40, 0x0, 0x20])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    cs = bench.ClockSampler(_fake_torch())
+    assert cs.ok
+    deadline = time.monotonic() + 10.0
+    with cs:
+        while fake.calls < 8 and time.monotonic() < deadline:
+            time.sleep(0.001)
+    s = cs.summary()
+    assert s["sm_max_mhz"] == 1965
+    assert s["sm_mhz"] == 1965          # the median, not the mean or the minimum
+    # gpu_idle is dropped; every other bit seen in any sample is reported
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+    assert s["samples"] == len(cs.samples) >= 8
+
+
+def test_clock_sampler_without_nvml_reports_the_error(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml([], [], fail_init=True))
+    cs = bench.ClockSampler(_fake_torch())
+    with cs:
+        pass
+    s = cs.summary()
+    assert not cs.ok and s["sm_mhz"] is None and s["reasons"] == []
+    assert "NVML Shared Library Not Found" in s["error"]
+
+
+def test_measured_peak_and_fallback(monkeypatch, tmp_path):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (6650.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6537.5}))
+    assert bench.measured_peaks() == (6537.5, "measured")
+
+
+def test_recorded_traffic_only_for_the_captured_source(monkeypatch, tmp_path):
+    csrc = tmp_path / "affine_group_quantized_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("qmv_b4", "decode_sweep") is None
+    h = bench.source_hash()
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"decode_sweep": {"qmv_b4": {"source_hash": h,
+                                     "dram_bytes_per_launch": 33067008}}}))
+    assert bench.recorded_traffic("qmv_b4", "decode_sweep") == 33067008
+    assert bench.recorded_traffic("qmv_b8", "decode_sweep") is None
+    (csrc / "k.cu").write_text("kernel v2\n")           # source changed since
+    assert bench.source_hash() != h
+    assert bench.recorded_traffic("qmv_b4", "decode_sweep") is None
+
+
+def test_committed_traffic_names_known_launches():
+    # every recorded entry belongs to a launch label of the workload it is
+    # filed under, so the bench's lookup by (label, workload) can find it
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    recorded = {k: v for k, v in d.items() if not k.startswith("_")}
+    assert recorded
+    for name, entries in recorded.items():
+        if name == "batched":   # its launch labels, without building its inputs
+            labels = {f"qmv_M{M}_gs{gs}" for M in (1, 2, 4, 8) for gs in (32, 128)}
+        else:
+            labels = {l.label for l in bench.workload(name)[0]}
+        assert set(entries) <= labels, name
+        for e in entries.values():
+            assert e["dram_bytes_per_launch"] > 0 and len(e["source_hash"]) == 16
