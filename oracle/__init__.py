@@ -45,6 +45,10 @@ def lib() -> ctypes.CDLL:
                                              P, I, P, P, I]
         L.oracle_gather.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I,
                                     P, P, P, I]
+        L.oracle_bf16_round.restype = ctypes.c_uint16
+        L.oracle_bf16_round.argtypes = [ctypes.c_double, ctypes.c_double]
+        L.oracle_dequantize_bf16.argtypes = [P, P, P, I, I, I, I, P]
+        L.oracle_affine_quantize.argtypes = [P, I, I, I, I, P, P, P]
         _lib = L
     return _lib
 
@@ -147,3 +151,31 @@ def gather(x, w, scales, biases, lhs, rhs, num_pairs, num_x_rows, E, N, K,
     if rc < 0:
         raise ValueError("oracle_gather: bad arguments")
     return y, a, valid
+
+
+def bf16_round(hi: float, lo: float = 0.0) -> int:
+    """bf16 bit pattern nearest to the exact sum hi + lo (ties to even)."""
+    return int(lib().oracle_bf16_round(float(hi), float(lo)))
+
+
+def dequantize_bf16(w, scales, biases, N, K, bits, gs):
+    """bf16 [N, K] bit patterns of scale * q + bias, rounded once."""
+    w, s, b = _c(w, np.uint32), _c(scales, np.uint16), _c(biases, np.uint16)
+    out = np.zeros((N, K), dtype=np.uint16)
+    if lib().oracle_dequantize_bf16(_p(w), _p(s), _p(b), N, K, bits, gs,
+                                    _p(out)):
+        raise ValueError("oracle_dequantize_bf16: bad arguments")
+    return out
+
+
+def affine_quantize(w, N, K, bits, gs):
+    """bf16 [N, K] weights -> (packed uint32 [N, K*bits/32], bf16 scales
+    [N, K/gs], bf16 biases [N, K/gs]), computed in binary32."""
+    w = _c(w, np.uint16)
+    wq = np.zeros((N, K * bits // 32), dtype=np.uint32)
+    s = np.zeros((N, K // gs), dtype=np.uint16)
+    b = np.zeros((N, K // gs), dtype=np.uint16)
+    if lib().oracle_affine_quantize(_p(w), N, K, bits, gs, _p(wq), _p(s),
+                                    _p(b)):
+        raise ValueError("oracle_affine_quantize: bad arguments")
+    return wq, s, b

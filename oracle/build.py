@@ -1,7 +1,8 @@
 """Build the CPU oracle (oracle.c -> liboracle.so) with gcc.
 
 Test infrastructure: the product library never links this.  Compiled with
--O2 and without -ffast-math so that fp64 arithmetic follows IEEE order.
+-O2, without -ffast-math and without contraction into fused multiply-adds,
+so that fp64 and fp32 arithmetic follow IEEE order, one rounding per operation.
 """
 import os
 import subprocess
@@ -18,7 +19,7 @@ def build(force: bool = False) -> str:
     ):
         return LIB
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
-           "-fno-fast-math", "-Wall", "-Wextra", "-o", LIB, SRC, "-lm"]
+           "-fno-fast-math", "-ffp-contract=off", "-Wall", "-Wextra", "-o", LIB, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     return LIB
 

@@ -9,11 +9,14 @@
  *
  * Every result is computed in IEEE double precision, element by element, in
  * the order the definitions state.  No blocking, no reordering, no fusion.
+ * The one exception is the quantizer, whose codes the pages decide in
+ * binary32: it follows that precision operation by operation.
  *
  * Sources (web pages, cited by page title and section):
  *   [MLX-Q]  "mlx/include/mlx/backend/metal/kernels/quantized.h" (MLX 0.30.1),
- *            pack factor / bytes-per-pack helpers, affine_dequantize kernel,
- *            qdot, adjust_matrix_offsets (gather form), affine_gather_qmm_rhs.
+ *            pack factor / bytes-per-pack helpers, affine_quantize and
+ *            affine_dequantize kernels, qdot, adjust_matrix_offsets (gather
+ *            form), affine_gather_qmm_rhs.
  *   [MLX-OPS] "Get trellis to run" compare page, mlx/ops.cpp
  *            extract_quantized_matmul_dims (shape rules).
  *   [GQMM]   "mlx.core.gather_qmm" API page (lhs_indices / rhs_indices,
@@ -342,4 +345,172 @@ int oracle_gather(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
         if (rc) return -1;
     }
     return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Producer side of the format: affine_quantize and affine_dequantize        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The bf16 value nearest to the exact sum hi + lo, ties to even, where hi and
+ * lo are doubles with |lo| at most half an ulp of hi (the pair a two-sum
+ * produces; lo == 0 for a single double).  bf16 keeps 8 significant bits and
+ * the binary32 exponent range: below 2^-126 its spacing is fixed at 2^-133;
+ * results of magnitude 2^128 and above overflow to infinity.
+ *
+ * hi is scaled by its bf16 spacing (a power of two, so exactly) and rounded
+ * to an integer.  Because hi has at most 53 significant bits and lies on the
+ * binary64 grid, the exact sum can only round differently from hi itself when
+ * hi sits exactly halfway between two bf16 values; lo then decides.
+ * Pins: brute force against exact rational rounding (ties, subnormals,
+ * overflow included) in the test suite.
+ */
+uint16_t oracle_bf16_round(double hi, double lo)
+{
+    if (isnan(hi)) return 0x7fc0;
+    if (isinf(hi)) return hi > 0 ? 0x7f80 : 0xff80;
+    double r;
+    if (hi == 0.0) {
+        r = hi;
+    } else {
+        int e;
+        frexp(hi, &e);                     /* 2^(e-1) <= |hi| < 2^e */
+        int ue = e - 8 > -133 ? e - 8 : -133;
+        double q = ldexp(hi, -ue);         /* exact */
+        double fl = floor(q);
+        double frac = q - fl;              /* exact */
+        double n;
+        if (frac > 0.5 || (frac == 0.5 && lo > 0.0)) n = fl + 1.0;
+        else if (frac < 0.5 || (frac == 0.5 && lo < 0.0)) n = fl;
+        else n = fmod(fl, 2.0) == 0.0 ? fl : fl + 1.0;   /* exact tie: even */
+        r = ldexp(n, ue);
+        if (r == 0.0) r = copysign(0.0, hi);
+    }
+    if (fabs(r) >= 0x1p128) return r > 0 ? 0x7f80 : 0xff80;
+    float f = (float)r;                    /* exact: 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+static float bf16_to_float(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * Dequantize to bf16: out[n][k] = bf16(scale * q + bias), the affine map of
+ * [MLX-Q] affine_dequantize, with the exact value rounded once to bf16 (ties
+ * to even).  scale * q is exact in double (8 by 8 significant bits); the sum
+ * with the bias is carried as a two-sum pair so the rounding is exact for any
+ * exponents.
+ * Pins: brute force with exact rationals; agreement with oracle_dequant
+ * (the fp64 w_hat) wherever that is exact.
+ */
+int oracle_dequantize_bf16(const uint32_t *w, const uint16_t *scales,
+                           const uint16_t *biases, int N, int K, int bits,
+                           int gs, uint16_t *out)
+{
+    if (oracle_check_shape(N, K, bits, gs)) return -1;
+    const long long rb = oracle_row_bytes(K, bits);
+    const long long G = K / gs;
+    for (long long n = 0; n < N; ++n) {
+        const uint8_t *row = (const uint8_t *)w + n * rb;
+        for (long long k = 0; k < K; ++k) {
+            double a = oracle_bf16_to_double(scales[n * G + k / gs]) *
+                       (double)code_at(row, k, bits);
+            double b = oracle_bf16_to_double(biases[n * G + k / gs]);
+            double s = a + b;              /* Knuth's two-sum: s + e == a + b */
+            double bv = s - a;
+            double av = s - bv;
+            double e = (a - av) + (b - bv);
+            out[n * K + k] = oracle_bf16_round(s, e);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Quantize one group of gs weights, in binary32 as [MLX-Q] affine_quantize
+ * computes it (the codes are decided in that precision):
+ *   w_min starts at the largest finite bf16 and w_max at 0, then take the
+ *   group's min and max (so w_max = max(0, max w));
+ *   delta = max((w_max - w_min) / n_bins, 1e-7), n_bins = 2^bits - 1;
+ *   the edge is the endpoint of larger magnitude (w_min when
+ *   |w_min| > |w_max|, else w_max); the scale is +delta for the w_min edge
+ *   and -delta for the w_max edge;
+ *   q0 = round(edge / scale) (halves away from zero); unless q0 == 0 the scale
+ *   becomes edge / q0 and the bias the edge itself (so the edge is code 0 and
+ *   zero is code -q0), else the bias is 0;
+ *   code = min(round((w - bias) / scale), n_bins).
+ * scale and bias are stored as bf16 (round to nearest even); the codes use
+ * the binary32 values.
+ * Pins: hand-derived groups (tests/golden/quantize.txt); code 0 at the edge;
+ * codes monotone in w; reconstruction within the rounding bound.
+ */
+static void quantize_group(const uint16_t *w, int gs, int bits, uint8_t *q,
+                           uint16_t *scale_out, uint16_t *bias_out)
+{
+    const float n_bins = (float)((1 << bits) - 1);
+    const float eps = 1e-7f;
+    float w_min = bf16_to_float(0x7f7f);   /* largest finite bf16 */
+    float w_max = 0.0f;
+    for (int i = 0; i < gs; ++i) {
+        float v = bf16_to_float(w[i]);
+        w_min = fminf(w_min, v);
+        w_max = fmaxf(w_max, v);
+    }
+    float scale = fmaxf((w_max - w_min) / n_bins, eps);
+    int side = fabsf(w_min) > fabsf(w_max);
+    scale = side ? scale : -scale;
+    float edge = side ? w_min : w_max;
+    float q0 = roundf(edge / scale);
+    int at_zero = q0 == 0.0f;
+    scale = at_zero ? scale : edge / q0;
+    float bias = at_zero ? 0.0f : edge;
+    *scale_out = oracle_bf16_round((double)scale, 0.0);
+    *bias_out = oracle_bf16_round((double)bias, 0.0);
+    for (int i = 0; i < gs; ++i) {
+        float v = bf16_to_float(w[i]);
+        float c = fminf(roundf((v - bias) / scale), n_bins);
+        q[i] = (uint8_t)c;
+    }
+}
+
+/* Write code k of a packed row, one bit at a time (the layout code_at reads). */
+static void put_code(uint8_t *row, long long k, int bits, unsigned q)
+{
+    for (int b = 0; b < bits; ++b) {
+        long long bit = k * bits + b;
+        uint8_t m = (uint8_t)(1u << (bit & 7));
+        if ((q >> b) & 1u) row[bit >> 3] |= m;
+        else row[bit >> 3] &= (uint8_t)~m;
+    }
+}
+
+/*
+ * Quantize a bf16 [N, K] matrix: packed codes [N, K*bits/32] (the row layout
+ * above), bf16 scales and biases [N, K/gs].  Groups are gs consecutive
+ * elements of a row ([MLX-Q] affine_quantize indexes groups by element / gs
+ * over the flattened matrix, which is the same thing when gs divides K).
+ */
+int oracle_affine_quantize(const uint16_t *w, int N, int K, int bits, int gs,
+                           uint32_t *wq, uint16_t *scales, uint16_t *biases)
+{
+    if (oracle_check_shape(N, K, bits, gs)) return -1;
+    const long long rb = oracle_row_bytes(K, bits);
+    const long long G = K / gs;
+    uint8_t q[128];
+    for (long long n = 0; n < N; ++n) {
+        uint8_t *row = (uint8_t *)wq + n * rb;
+        for (long long g = 0; g < G; ++g) {
+            quantize_group(w + n * K + g * gs, gs, bits, q, &scales[n * G + g],
+                           &biases[n * G + g]);
+            for (int i = 0; i < gs; ++i) put_code(row, g * gs + i, bits, q[i]);
+        }
+    }
+    return 0;
 }

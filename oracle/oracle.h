@@ -35,4 +35,10 @@ int oracle_gather(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
                   const uint32_t *rhs, int num_pairs, int num_x_rows, int E,
                   int N, int K, int bits, int gs, double *y, double *a,
                   int32_t *valid, int nthreads);
+uint16_t oracle_bf16_round(double hi, double lo);
+int oracle_dequantize_bf16(const uint32_t *w, const uint16_t *scales,
+                           const uint16_t *biases, int N, int K, int bits,
+                           int gs, uint16_t *out);
+int oracle_affine_quantize(const uint16_t *w, int N, int K, int bits, int gs,
+                           uint32_t *wq, uint16_t *scales, uint16_t *biases);
 #endif
