@@ -165,7 +165,7 @@ def _golden_groups():
 
 def test_quantize_golden_groups():
     cases = _golden_groups()
-    assert len(cases) == 10
+    assert len(cases) == 12
     for c in cases:
         gs, bits = c["gs"], c["bits"]
         vals = c["lead"] + [c["fill"]] * (gs - len(c["lead"]))
