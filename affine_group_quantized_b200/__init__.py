@@ -64,12 +64,19 @@ def lib() -> ctypes.CDLL:
         L.qmv_last_error.argtypes = []
         L.qmv_abi_version.restype = I
         L.qmv_abi_version.argtypes = []
+        L.affine_quantize.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.affine_dequantize.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.affine_quantize.restype = I
+        L.affine_dequantize.restype = I
+        L.qmv_quant_last_error.restype = ctypes.c_char_p
+        L.qmv_quant_last_error.argtypes = []
         _lib = L
     return _lib
 
 
 EXPORTED = ("qmv", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
-            "qmv_last_error", "qmv_abi_version")
+            "qmv_last_error", "qmv_abi_version", "affine_quantize",
+            "affine_dequantize", "qmv_quant_last_error")
 
 
 def _ptr(a):
@@ -92,6 +99,11 @@ def _stream(stream):
 def _check(func: str, rc: int):
     if rc != QMV_OK:
         raise QmvError(func, rc, lib().qmv_last_error().decode())
+
+
+def _check_quant(func: str, rc: int):
+    if rc != QMV_OK:
+        raise QmvError(func, rc, lib().qmv_quant_last_error().decode())
 
 
 def last_error() -> str:
@@ -141,3 +153,18 @@ def gather_qmv(x, w, scales, biases, lhs_indices, rhs_indices, y, num_pairs,
         _ptr(rhs_indices), _ptr(y), num_pairs, num_x_rows, num_experts, N, K,
         bits, group_size, 1 if sorted_indices else 0, _ptr(d_status),
         _stream(stream)))
+
+
+def affine_quantize(w, w_q, scales, biases, N, K, bits, group_size, stream=None):
+    """Quantize bf16 w[N,K] into packed w_q and bf16 scales/biases [N,K/gs]."""
+    _check_quant("affine_quantize", lib().affine_quantize(
+        _ptr(w), _ptr(w_q), _ptr(scales), _ptr(biases), N, K, bits, group_size,
+        _stream(stream)))
+
+
+def affine_dequantize(w_q, scales, biases, w_hat, N, K, bits, group_size,
+                      stream=None):
+    """w_hat[N,K] = bf16(scale * q + bias) from the packed format."""
+    _check_quant("affine_dequantize", lib().affine_dequantize(
+        _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(w_hat), N, K, bits,
+        group_size, _stream(stream)))

@@ -171,7 +171,61 @@ int gather_qmv(const void *x, const uint32_t *w, const void *scales,
                int group_size, int sorted_indices, int *d_status,
                void *stream);
 
-/* Message for the last non-OK return on this thread ("" if none). */
+/*
+ * affine_quantize -- quantize a bf16 matrix into the packed format above.
+ *
+ * Defined by the pages' affine_quantize kernel ("mlx/include/mlx/backend/
+ * metal/kernels/quantized.h", MLX 0.30.1).  For each group of group_size
+ * consecutive elements of a row, in binary32:
+ *   w_min = min(largest finite bf16, group), w_max = max(0, group);
+ *   delta = max((w_max - w_min) / n_bins, 1e-7), n_bins = 2^bits - 1;
+ *   edge = w_min and scale = +delta if |w_min| > |w_max|,
+ *   else edge = w_max and scale = -delta;
+ *   q0 = round(edge / scale) (halves away from zero);
+ *   if q0 != 0: scale = edge / q0, bias = edge; else bias = 0;
+ *   code = min(round((w - bias) / scale), n_bins).
+ * The codes are decided with the binary32 scale and bias; the stored scale
+ * and bias are those values rounded to bf16 (nearest, ties to even), so the
+ * bias is the group's edge exactly.  Every division is IEEE binary32
+ * (correctly rounded), so codes, scales and biases are bit-identical to the
+ * same steps run on any IEEE host.  Inputs must be finite; groups whose
+ * values all lie within n_bins * 1e-7 of each other and exceed 1e31 in
+ * magnitude overflow q0 and are outside the definition.
+ *   w        bf16 [N, K] (read)
+ *   w_q      uint32 [N, K*bits/32] (written; the row layout above)
+ *   scales   bf16 [N, K/group_size] (written)
+ *   biases   bf16 [N, K/group_size] (written)
+ * N >= 0 (N = 0 enqueues nothing), K a positive multiple of group_size.
+ * Outputs must not overlap the input.  One kernel launch; no allocation.
+ * On error qmv_quant_last_error() describes the failure.
+ */
+int affine_quantize(const void *w, uint32_t *w_q, void *scales, void *biases,
+                    int N, int K, int bits, int group_size, void *stream);
+
+/*
+ * affine_dequantize -- expand packed codes to bf16 weights:
+ *   w_hat[n][k] = bf16(scale[n][g] * q[n][k] + bias[n][g]),  g = k / group_size
+ *
+ * Defined by the pages' affine_dequantize kernel (same page).  The exact value
+ * scale * q + bias is rounded once to bf16 (nearest, ties to even), for any
+ * scale and bias with |scale * q| < 2^128.
+ *   w_q              uint32 [N, K*bits/32] (read; the row layout above)
+ *   scales, biases   bf16 [N, K/group_size] (read)
+ *   w_hat            bf16 [N, K] (written; must not overlap the inputs)
+ * N >= 0 (N = 0 enqueues nothing), K a positive multiple of group_size.
+ * One kernel launch; no allocation.  On error qmv_quant_last_error()
+ * describes the failure.
+ */
+int affine_dequantize(const uint32_t *w_q, const void *scales,
+                      const void *biases, void *w_hat, int N, int K, int bits,
+                      int group_size, void *stream);
+
+/* Message for the last non-OK return of affine_quantize or
+ * affine_dequantize on this thread ("" if none). */
+const char *qmv_quant_last_error(void);
+
+/* Message for the last non-OK return of the other entry points on this
+ * thread ("" if none). */
 const char *qmv_last_error(void);
 
 /* ABI version of this header (incremented on incompatible change). */

@@ -30,7 +30,9 @@ def declared_functions():
 def test_header_lists_the_entry_points():
     names = declared_functions()
     assert {"qmv", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
-            "qmv_last_error", "qmv_abi_version"} <= set(names)
+            "qmv_last_error", "qmv_abi_version", "affine_quantize",
+            "affine_dequantize", "qmv_quant_last_error"} <= set(names)
+    assert set(agq.EXPORTED) <= set(names)
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -126,3 +128,53 @@ def test_binding_raises_with_message(lib):
         agq.qmv(A, A, A, A, A, 1, 64, 100, 4, 64, stream=0)
     assert ei.value.status == agq.QMV_ERR_SHAPE
     assert "group_size" in str(ei.value)
+
+
+def test_quantize_argument_checks(lib):
+    f = lib.affine_quantize
+    # w w_q scales biases N K bits gs stream
+    base = [A, A, A, A, 4, 128, 4, 64, None]
+
+    def call(i, v):
+        a = list(base); a[i] = v
+        return f(*a)
+
+    for i in range(4):
+        assert call(i, None) == agq.QMV_ERR_NULL
+    assert call(6, 7) == agq.QMV_ERR_UNSUPPORTED      # bits
+    assert call(7, 16) == agq.QMV_ERR_UNSUPPORTED     # group size
+    assert call(4, -1) == agq.QMV_ERR_SHAPE
+    assert call(5, 0) == agq.QMV_ERR_SHAPE
+    assert call(5, 96) == agq.QMV_ERR_SHAPE           # K % group_size
+    for i in range(4):
+        assert call(i, A + 8) == agq.QMV_ERR_ALIGN
+    assert call(4, 0) == agq.QMV_OK                   # empty: nothing enqueued
+    assert "" == agq.lib().qmv_quant_last_error().decode()
+
+
+def test_dequantize_argument_checks(lib):
+    f = lib.affine_dequantize
+    # w_q scales biases w_hat N K bits gs stream
+    base = [A, A, A, A, 4, 128, 4, 64, None]
+
+    def call(i, v):
+        a = list(base); a[i] = v
+        return f(*a)
+
+    for i in range(4):
+        assert call(i, None) == agq.QMV_ERR_NULL
+    assert call(6, 1) == agq.QMV_ERR_UNSUPPORTED
+    assert call(7, 256) == agq.QMV_ERR_UNSUPPORTED
+    assert call(5, 160) == agq.QMV_ERR_SHAPE
+    assert call(3, A + 2) == agq.QMV_ERR_ALIGN
+    assert call(4, 0) == agq.QMV_OK
+
+
+def test_quant_binding_raises_with_its_own_message(lib):
+    with pytest.raises(agq.QmvError) as ei:
+        agq.affine_quantize(A, A, A, A, 2, 100, 4, 64, stream=0)
+    assert ei.value.status == agq.QMV_ERR_SHAPE
+    assert "group_size" in str(ei.value)
+    with pytest.raises(agq.QmvError) as ei:
+        agq.affine_dequantize(A, A, A, A, 2, 128, 9, 64, stream=0)
+    assert ei.value.status == agq.QMV_ERR_UNSUPPORTED and "bits=9" in str(ei.value)

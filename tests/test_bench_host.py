@@ -138,7 +138,7 @@ def test_measured_peak_and_fallback(monkeypatch, tmp_path):
 def test_recorded_traffic_only_for_the_captured_source(monkeypatch, tmp_path):
     csrc = tmp_path / "affine_group_quantized_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cu").write_text("kernel v1\n")
+    (csrc / "qmv_stream.cuh").write_text("kernel v1\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.recorded_traffic("qmv_b4", "decode_sweep") is None
     h = bench.source_hash()
@@ -148,7 +148,10 @@ def test_recorded_traffic_only_for_the_captured_source(monkeypatch, tmp_path):
                                      "dram_bytes_per_launch": 33067008}}}))
     assert bench.recorded_traffic("qmv_b4", "decode_sweep") == 33067008
     assert bench.recorded_traffic("qmv_b8", "decode_sweep") is None
-    (csrc / "k.cu").write_text("kernel v2\n")           # source changed since
+    (csrc / "qmv_quant.cu").write_text("other kernels\n")   # not a GEMV source
+    assert bench.source_hash() == h
+    assert bench.recorded_traffic("qmv_b4", "decode_sweep") == 33067008
+    (csrc / "qmv_stream.cuh").write_text("kernel v2\n")     # source changed since
     assert bench.source_hash() != h
     assert bench.recorded_traffic("qmv_b4", "decode_sweep") is None
 
