@@ -36,24 +36,22 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) {
 // Dequantize: out = bf16(scale * q + bias), the exact value rounded once
 // ---------------------------------------------------------------------------
 
-// scale * q is exact in binary32 (8 by 8 significant bits).  The sum with the
-// bias is rounded once to binary32 (r) and its exact error recovered with a
-// two-sum (e).  r then rounds to bf16 exactly as the exact sum would, except
-// when r lies exactly halfway between two bf16 values and e != 0: there the
-// exact sum lies on e's side of r.
-__device__ __forceinline__ uint16_t affine_to_bf16(float q, float s, float b) {
+// scale * q is exact in binary32 (8 by 8 significant bits), so one fused
+// multiply-add rounds the exact scale * q + bias once to binary32 (r).  r
+// rounds to bf16 exactly as the exact sum would, except when r lies exactly
+// halfway between two bf16 values (its low 16 bits are 0x8000) while the sum
+// was not exact: there the exact sum lies on the side of the two-sum error e,
+// which the rare slow path recovers.
+__device__ __noinline__ uint16_t affine_tie_to_bf16(float q, float s, float b, float r) {
   const float p = __fmul_rn(q, s);
-  const float r = __fadd_rn(p, b);
   const float bv = __fsub_rn(r, p);
   const float av = __fsub_rn(r, bv);
   const float e = __fadd_rn(__fsub_rn(p, av), __fsub_rn(b, bv));
   const uint32_t u = __float_as_uint(r);
-  if ((u & 0xffffu) == 0x8000u && e != 0.0f) {
-    // sign-magnitude: adding 1 to the upper half grows the magnitude
-    const bool away = (e > 0.0f) == (r > 0.0f);
-    return static_cast<uint16_t>((u >> 16) + (away ? 1u : 0u));
-  }
-  return __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  if (e == 0.0f) return __bfloat16_as_ushort(__float2bfloat16_rn(r));  // a true tie
+  // sign-magnitude: adding 1 to the upper half grows the magnitude
+  const bool away = (e > 0.0f) == (r > 0.0f);
+  return static_cast<uint16_t>((u >> 16) + (away ? 1u : 0u));
 }
 
 template <int BITS>
@@ -78,14 +76,33 @@ affine_dequantize_kernel(const uint32_t *__restrict__ wq,
     const long long g = (c * 8) >> gs_shift;
     const float s = bf16_bits_to_float(__ldg(scales + g));
     const float b = bf16_bits_to_float(__ldg(biases + g));
-    uint32_t h[8];
+    float q[8], r[8];
+    bool tie = false;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float q = static_cast<float>(static_cast<uint32_t>(v >> (BITS * i)) & kMask);
-      h[i] = affine_to_bf16(q, s, b);
+      // the code as an exact float: 2^23 + q has q in its low mantissa bits
+      const uint32_t code = static_cast<uint32_t>(v >> (BITS * i)) & kMask;
+      q[i] = __fsub_rn(__uint_as_float(0x4b000000u | code), 8388608.0f);
+      r[i] = __fmaf_rn(q[i], s, b);
+      tie |= (__float_as_uint(r[i]) & 0xffffu) == 0x8000u;
     }
-    out[c] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
-                        h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
+      h[j] = *reinterpret_cast<const uint32_t *>(&pr);
+    }
+    if (tie) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((__float_as_uint(r[i]) & 0xffffu) == 0x8000u) {
+          const uint32_t hi = affine_tie_to_bf16(q[i], s, b, r[i]);
+          const int sh = 16 * (i & 1);
+          h[i >> 1] = (h[i >> 1] & ~(0xffffu << sh)) | (hi << sh);
+        }
+      }
+    }
+    out[c] = make_uint4(h[0], h[1], h[2], h[3]);
   }
 }
 
