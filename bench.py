@@ -45,6 +45,12 @@ def qmv_bytes(M, N, K, bits, gs):
     return N * K * bits // 8 + 2 * 2 * N * (K // gs) + 2 * M * K + 2 * M * N
 
 
+def quant_bytes(N, K, bits, gs):
+    """Bytes one quantize (or dequantize) of an [N, K] matrix moves: the bf16
+    matrix, the packed codes, and the bf16 scales and biases."""
+    return 2 * N * K + N * K * bits // 8 + 2 * 2 * N * (K // gs)
+
+
 class Launch:
     """One kernel launch of a step: label, algorithmic bytes, host inputs."""
 
@@ -109,6 +115,19 @@ def workload(name):
                             sorted=srt == "sorted"))
         cfg = {"workload": "MoE gather_qmv", "experts": E, "N": N, "K": K, "bits": bits,
                "group_size": gs, "tokens": T, "top_k": k, "touched_experts": touched}
+    elif name == "quantize":
+        # the producer side of the format on the decode weight shape: one
+        # quantize of a bf16 matrix and one dequantize of a packed matrix
+        N, K, bits, gs = 14336, 4096, 4, 64
+        w = synth.normal_bf16((N, K), seed=6000)
+        _, wq, s, b = synth.qmv_inputs(1, N, K, bits, gs, seed=6001)
+        nb = quant_bytes(N, K, bits, gs)
+        L.append(Launch(f"quantize_b{bits}", "quantize", nb, N=N, K=K, bits=bits, gs=gs,
+                        w=w))
+        L.append(Launch(f"dequantize_b{bits}", "dequantize", nb, N=N, K=K, bits=bits,
+                        gs=gs, w=wq, s=s, b=b))
+        cfg = {"workload": "affine quantize + dequantize", "N": N, "K": K,
+               "group_size": gs, "bits": bits}
     else:
         raise SystemExit(f"unknown workload {name}")
     return L, cfg
@@ -497,6 +516,168 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_quant(args):
+    """GPU arm of the quantize workload: one step = affine_quantize of a bf16
+    matrix and affine_dequantize of a packed one.  Inputs rotate through
+    copies so that more than twice the L2 capacity streams between two reads
+    of the same bytes; the dequantize of step k reads the codes the quantize
+    of an earlier step wrote (copy k + 1), so it never reads L2-hot output."""
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import affine_group_quantized_b200 as agq
+    agq.lib()
+
+    launches, cfg = workload("quantize")
+    lq, ld = launches
+    N, K, bits, gs = lq.N, lq.K, lq.bits, lq.gs
+    step_bytes = lq.nbytes + ld.nbytes
+    copies = max(3, -(-2 * L2_BYTES // (2 * N * K)) + 1)
+    bf, i32, i16 = torch.bfloat16, torch.int32, torch.int16
+    W = [_dev(lq.w, torch) for _ in range(copies)]
+    Q = [_dev(ld.w, torch) for _ in range(copies)]
+    S = [_dev(ld.s, torch) for _ in range(copies)]
+    B = [_dev(ld.b, torch) for _ in range(copies)]
+    Y = torch.empty((N, K), dtype=bf, device="cuda")
+
+    def quant(k):
+        c = k % copies
+        agq.affine_quantize(W[c], Q[c], S[c], B[c], N, K, bits, gs)
+
+    def dequant(k):
+        c = (k + 1) % copies
+        agq.affine_dequantize(Q[c], S[c], B[c], Y, N, K, bits, gs)
+
+    def step(k):
+        quant(k)
+        dequant(k)
+
+    for k in range(max(args.warmup, copies)):
+        step(k)
+    torch.cuda.synchronize()
+    graphs = []
+    for c in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(c)
+        graphs.append(g)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    Ks = args.steps
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch)
+    torch.cuda.synchronize()
+    with sampler:
+        t0.record(stream)
+        for k in range(Ks):
+            graphs[k % copies].replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
+
+    # each kernel alone: a graph of 3 * copies back-to-back launches
+    dur = []
+    for fn in (quant, dequant):
+        R = 3 * copies
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(R):
+                fn(r)
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(1, min(100, 2 * Ks // R))
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        dur.append(a.elapsed_time(b_) / (reps * R))
+
+    # end to end: the bf16 matrix in from pinned host memory, quantize,
+    # dequantize the result, and the packed matrix and the bf16 round trip out
+    hw = W[0].detach().cpu().pin_memory()
+    outs = (Q[0], S[0], B[0], Y)
+    houts = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+    h2d = hw.numel() * hw.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+
+    def e2e_step():
+        W[0].copy_(hw, non_blocking=True)
+        agq.affine_quantize(W[0], Q[0], S[0], B[0], N, K, bits, gs)
+        agq.affine_dequantize(Q[0], S[0], B[0], Y, N, K, bits, gs)
+        for h, d in zip(houts, outs):
+            h.copy_(d, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    eg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(eg):
+        e2e_step()
+    eg.replay()
+    torch.cuda.synchronize()
+    ek = max(3, min(Ks, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ek):
+        eg.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
+    del graphs, eg
+
+    peak, peak_kind = measured_peaks()
+    per = {}
+    for l, d in zip(launches, dur):
+        gbs = l.nbytes / (d * 1e-3) / 1e9
+        per[l.label] = {"us": round(d * 1e3, 3), "GB/s": round(gbs, 1),
+                        "frac_of_measured_peak": round(gbs / peak, 4), "bytes": l.nbytes}
+    dom = 0 if dur[0] >= dur[1] else 1
+    ach = launches[dom].nbytes / (dur[dom] * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(job_gbs(world, step_bytes, Ks, ms), 1),
+        "unit": UNIT, "n_gpus": world, "steps": Ks, "warmup": args.warmup,
+        "ms_per_step": round(ms / Ks, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (bf16 in/out)", "data": "synthetic",
+        "config": dict(cfg, l2=f"inputs larger than L2: {copies} rotating copies of every "
+                               f"input; dequantize reads codes written one step earlier",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       graphs="timed steps replayed as one CUDA graph per step"),
+        "roofline": {"bound": "hbm", "kernel": launches[dom].label, "achieved": round(ach, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+                     "peak_kind": peak_kind,
+                     "traffic": recorded_traffic(launches[dom].label, "quantize"),
+                     "algorithmic_bytes_per_launch": launches[dom].nbytes},
+        "per_launch": per,
+        "e2e": {"value": round(job_gbs(world, step_bytes, ek, e2e_ms), 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "bf16 matrix copied in, packed matrix and round trip copied out "
+                        "every step; each step replayed as one CUDA graph"},
+        "gpu_launches": 2 * Ks,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(launches, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle arm (reference) and CPU baseline
 # ---------------------------------------------------------------------------
@@ -519,6 +700,21 @@ def _oracle_launch(l, rows, nthreads):
     elif l.kind == "gather":
         oracle.gather(l.x, l.w, l.s, l.b, l.lhs, l.rhs, l.P, l.T, l.E, l.N, l.K,
                       l.bits, l.gs, nthreads=nthreads)
+    elif l.kind == "quantize":
+        n = l.N if rows is None else len(rows)
+        oracle.affine_quantize(l.w[:n], n, l.K, l.bits, l.gs)
+    elif l.kind == "dequantize":
+        n = l.N if rows is None else len(rows)
+        oracle.dequantize_bf16(l.w[:n], l.s[:n], l.b[:n], n, l.K, l.bits, l.gs)
+
+
+QUANT_KINDS = ("quantize", "dequantize")
+
+
+def _threads_used(launches, nthreads):
+    """The oracle's GEMVs run on `nthreads` threads; its quantizer and
+    dequantizer on one."""
+    return 1 if all(l.kind in QUANT_KINDS for l in launches) else nthreads
 
 
 def _sample(l, frac):
@@ -555,11 +751,12 @@ def cpu_baseline(launches, budget_s=20.0, frac=None):
             nb += b
         passes += 1
     dt = time.perf_counter() - t
-    return {"value": round(nb / dt / 1e9, 4), "unit": UNIT, "cores": nthreads,
+    return {"value": round(nb / dt / 1e9, 4), "unit": UNIT,
+            "cores": _threads_used(launches, nthreads),
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"{passes} pass(es) over the first {frac:.3f} of the rows of "
-                      f"every launch of one step (gather: all pairs), fp64 plain-C "
-                      f"oracle, {nthreads} threads"}
+                      f"every launch of one step (gather: all pairs), plain-C "
+                      f"oracle, {_threads_used(launches, nthreads)} thread(s)"}
 
 
 def run_reference(args):
@@ -587,8 +784,10 @@ def run_reference(args):
            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(args.steps, 1), 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "f64", "data": "synthetic", "config": cfg, "impl": "reference",
-           "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": nthreads,
+           "dtype": "f32 quantize, f64 dequantize" if args.workload == "quantize" else "f64",
+           "data": "synthetic", "config": cfg, "impl": "reference",
+           "cpu_baseline": {"value": round(value, 4), "unit": UNIT,
+                            "cores": _threads_used(launches, nthreads),
                             "kind": "oracle",
                             "sample": f"first {frac:.3f} of the rows of every launch per "
                                       f"step (gather: all pairs)"},
@@ -606,7 +805,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_sweep",
                     choices=["decode_sweep", "qmv_small", "ffn_int8", "batched",
-                             "moe_gather"])
+                             "moe_gather", "quantize"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
@@ -614,6 +813,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "quantize":
+        run_quant(args)
     else:
         run_ours(args)
 

@@ -38,6 +38,16 @@ def test_ffn_bytes_are_the_arrays_read_and_written():
                            2 * 2 * silu.K + 2 * silu.N)
 
 
+def test_quantize_bytes_are_the_matrix_and_its_packed_form():
+    quant, dequant = bench.workload("quantize")[0]
+    bf16_matrix = 2 * quant.N * quant.K
+    for l in (quant, dequant):
+        # one side is the bf16 matrix, the other the codes, scales and biases
+        assert l.nbytes == bf16_matrix + _arrays_bytes(dequant.w, dequant.s, dequant.b)
+    assert quant.w.nbytes == bf16_matrix
+    assert bench._threads_used([quant, dequant], 8) == 1
+
+
 def test_gather_bytes_count_touched_experts_only():
     launches, cfg = bench.workload("moe_gather")
     for l in launches:
