@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.oracle_bf16_round.argtypes = [ctypes.c_double, ctypes.c_double]
         L.oracle_dequantize_bf16.argtypes = [P, P, P, I, I, I, I, P]
         L.oracle_affine_quantize.argtypes = [P, I, I, I, I, P, P, P]
+        L.oracle_qvm.argtypes = [P, P, P, P, I, I, I, I, I, P, P]
         _lib = L
     return _lib
 
@@ -179,3 +180,14 @@ def affine_quantize(w, N, K, bits, gs):
                                     _p(b)):
         raise ValueError("oracle_affine_quantize: bad arguments")
     return wq, s, b
+
+
+def qvm(x, w, scales, biases, M, K, N, bits, gs):
+    """y[M, N] = x[M, K] @ dequant(w) for a packed w of K rows of N codes
+    (scales/biases [K, N/gs]); returns (y, a) as qmv does."""
+    x, w = _c(x, np.uint16), _c(w, np.uint32)
+    s, b = _c(scales, np.uint16), _c(biases, np.uint16)
+    y = np.zeros((M, N)); a = np.zeros((M, N))
+    if lib().oracle_qvm(_p(x), _p(w), _p(s), _p(b), M, K, N, bits, gs, _p(y), _p(a)):
+        raise ValueError("oracle_qvm: bad arguments")
+    return y, a

@@ -514,3 +514,45 @@ int oracle_affine_quantize(const uint16_t *w, int N, int K, int bits, int gs,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* qvm: the product with the non-transposed matrix                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * qvm: y[m][n] = sum_k x[m][k] * w_hat[k][n]   (x @ dequant(W), transpose false)
+ *
+ * [MLX-Q] qvm_impl: the packed matrix has K rows (the input length) of N
+ * codes (the output length), in the row layout above; its groups of gs run
+ * along each row, so w_hat[k][n] = scales[k][n / gs] * q[k][n] +
+ * biases[k][n / gs].  Each output sums its K terms in k order in fp64 and
+ * records sum_k |x * w_hat|.
+ * x bf16 [M, K]; w packed [K, N]; scales/biases bf16 [K, N/gs]; y, a [M, N].
+ * Pins: a dense fp64 matmul of the dequantized matrix; brute force on
+ * dyadic inputs (exact); equality with qmv of the transposed codes when the
+ * scales are constant over each block of gs rows.
+ */
+int oracle_qvm(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
+               const uint16_t *biases, int M, int K, int N, int bits, int gs,
+               double *y, double *a)
+{
+    if (M < 0 || oracle_check_shape(K, N, bits, gs)) return -1;
+    const long long rb = oracle_row_bytes(N, bits);
+    const long long G = N / gs;
+    for (long long m = 0; m < M; ++m) {
+        for (long long n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            for (long long k = 0; k < K; ++k) {
+                const uint8_t *row = (const uint8_t *)w + k * rb;
+                double t = oracle_bf16_to_double(x[m * K + k]) *
+                           w_hat_at(row, scales + k * G, biases + k * G, n,
+                                    bits, gs);
+                acc += t;
+                mag += fabs(t);
+            }
+            y[m * N + n] = acc;
+            a[m * N + n] = mag;
+        }
+    }
+    return 0;
+}

@@ -41,4 +41,7 @@ int oracle_dequantize_bf16(const uint32_t *w, const uint16_t *scales,
                            int gs, uint16_t *out);
 int oracle_affine_quantize(const uint16_t *w, int N, int K, int bits, int gs,
                            uint32_t *wq, uint16_t *scales, uint16_t *biases);
+int oracle_qvm(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
+               const uint16_t *biases, int M, int K, int N, int bits, int gs,
+               double *y, double *a);
 #endif
