@@ -11,8 +11,13 @@ formulations of the same layout (code i of a row sits at bits
 
 Tests build inputs from known codes with ``pack`` and compute expected values
 from the codes directly, so a layout mistake in the oracle cannot cancel.
+
+``exact_bf16`` rounds an exact rational (``fractions.Fraction``) to bf16, the
+reference for every rounding-to-bf16 check.
 """
 from __future__ import annotations
+
+from fractions import Fraction
 
 import numpy as np
 
@@ -56,3 +61,24 @@ def to_bf16_bits(v) -> np.ndarray:
     if np.any(f.astype(np.float64) != np.asarray(v, dtype=np.float64)):
         raise ValueError("value not exactly representable in fp32")
     return (u >> 16).astype(np.uint16)
+
+
+def exact_bf16(v: Fraction) -> int:
+    """bf16 bit pattern nearest to the rational v (ties to even)."""
+    if v == 0:
+        return 0
+    neg = v < 0
+    a = -v if neg else v
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1                                  # now 2^e <= a < 2^(e+1)
+    ue = max(e - 7, -133)                       # 8 significant bits
+    n = round(a / Fraction(2) ** ue)            # Fraction rounds half to even
+    r = n * Fraction(2) ** ue
+    if r >= Fraction(2) ** 128:
+        return 0xff80 if neg else 0x7f80
+    if r == 0:
+        return 0x8000 if neg else 0
+    u = int(np.array([float(r)], dtype=np.float32).view(np.uint32)[0])
+    assert u & 0xffff == 0
+    return (u >> 16) | (0x8000 if neg else 0)

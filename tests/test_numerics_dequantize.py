@@ -15,8 +15,7 @@ from fractions import Fraction
 
 import numpy as np
 
-from tests._codes import to_bf16_bits
-from tests.test_oracle_quantize_pins import _exact_bf16
+from tests._codes import exact_bf16 as _exact_bf16
 
 
 def _f32(x: Fraction) -> Fraction:

@@ -20,36 +20,15 @@ import numpy as np
 import pytest
 
 import oracle
-from tests._codes import bf16_value, pack, to_bf16_bits
+from tests._codes import bf16_value, exact_bf16 as _exact_bf16, pack, to_bf16_bits
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 ALL_BITS = (2, 3, 4, 5, 6, 8)
 
 
 # --------------------------------------------------------------------------
-# Exact rational reference for rounding to bf16
+# bf16 rounding
 # --------------------------------------------------------------------------
-
-def _exact_bf16(v: Fraction) -> int:
-    """bf16 bit pattern nearest to the rational v (ties to even)."""
-    if v == 0:
-        return 0
-    neg = v < 0
-    a = -v if neg else v
-    e = a.numerator.bit_length() - a.denominator.bit_length()
-    if Fraction(2) ** e > a:
-        e -= 1                                  # now 2^e <= a < 2^(e+1)
-    ue = max(e - 7, -133)                       # 8 significant bits
-    n = round(a / Fraction(2) ** ue)            # Fraction rounds half to even
-    r = n * Fraction(2) ** ue
-    if r >= Fraction(2) ** 128:
-        return 0xff80 if neg else 0x7f80
-    if r == 0:
-        return 0x8000 if neg else 0
-    u = int(np.array([float(r)], dtype=np.float32).view(np.uint32)[0])
-    assert u & 0xffff == 0
-    return (u >> 16) | (0x8000 if neg else 0)
-
 
 def _bf16_fraction(h: int) -> Fraction:
     return Fraction(float(bf16_value(np.uint16(h))))
