@@ -170,3 +170,26 @@ def test_empty_matrix_enqueues_nothing():
     agq.affine_dequantize(Q, S, B, Y, 0, 64, 4, 32)
     torch.cuda.synchronize()
     assert (Q == 7).all() and (S == 7).all() and (B == 7).all() and (Y == 0).all()
+
+
+@pytest.mark.parametrize("bits", (3, 4, 8))
+def test_quantized_weights_feed_qmv(bits):
+    # producer to consumer on the device: weights quantized by the kernel go
+    # straight into qmv; the oracle quantizes the same weights and runs its
+    # own qmv, and the two must agree within the GEMV tolerance
+    from affine_group_quantized_b200 import synth
+    from tests._parity import check, empty_bf16
+    N, K, gs = 300, 1024, 64
+    w = _weights(np.random.default_rng(70 + bits), N, K, "normal")
+    x = synth.normal_bf16((1, K), seed=71 + bits)
+    W = dev_bf16(w)
+    Q = torch.empty((N, K * bits // 32), dtype=torch.int32, device="cuda")
+    S = torch.empty((N, K // gs), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((N, K // gs), dtype=torch.bfloat16, device="cuda")
+    Y = empty_bf16(1, N)
+    agq.affine_quantize(W, Q, S, B, N, K, bits, gs)
+    agq.qmv(dev_bf16(x), Q, S, B, Y, 1, N, K, bits, gs)
+    torch.cuda.synchronize()
+    owq, os_, ob = oracle.affine_quantize(w, N, K, bits, gs)
+    y_ref, a_ref = oracle.qmv(x, owq, os_, ob, 1, N, K, bits, gs)
+    check(host_bits(Y), y_ref, a_ref, f"quantize -> qmv bits={bits}")
