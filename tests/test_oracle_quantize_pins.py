@@ -249,3 +249,46 @@ def test_quantize_rejects_bad_shapes():
         oracle.affine_quantize(w, 2, 64, 4, 48)      # group size
     with pytest.raises(ValueError):
         oracle.affine_quantize(w[:, :48], 2, 48, 4, 32)   # K % gs
+
+
+# --------------------------------------------------------------------------
+# Generated groups (hypothesis): zeros, subnormals, tiny spans, large values
+# --------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+_BF16_FINITE = st.integers(0, 0xFFFF).filter(lambda h: (h & 0x7F80) != 0x7F80)
+
+
+def _small_magnitude(h):
+    # finite and below 2^100 in magnitude (far inside the definition's range)
+    return ((h >> 7) & 0xFF) < 127 + 100
+
+
+@settings(max_examples=300, deadline=None)
+@given(bits=st.sampled_from(ALL_BITS),
+       vals=st.lists(_BF16_FINITE.filter(_small_magnitude), min_size=32, max_size=32),
+       base=_BF16_FINITE.filter(_small_magnitude),
+       spread=st.integers(0, 3))
+def test_quantize_generated_groups(bits, vals, base, spread):
+    gs = 32
+    if spread == 0:      # a near-constant group: every value within a few ulps of base
+        vals = [(base & 0xFF80) | (v & 0x3) for v in vals]
+    w = np.array([vals], dtype=np.uint16)
+    wq, s, b = oracle.affine_quantize(w, 1, gs, bits, gs)
+    q = oracle.unpack(wq, 1, gs, bits)[0].astype(np.int64)
+    x = bf16_value(w)[0]
+    n_bins = (1 << bits) - 1
+    lo, hi = x.min(), max(x.max(), 0.0)
+    edge = lo if abs(lo) > abs(hi) else hi
+    bias = bf16_value(b)[0, 0]
+    scale = bf16_value(s)[0, 0]
+    assert q.max() <= n_bins
+    assert bias == edge or bias == 0.0
+    if bias == 0.0 and edge != 0.0:
+        assert (q == 0).all()            # q0 rounded to 0: every code is 0
+    else:
+        assert (q[x == edge] == 0).all()
+    order = np.argsort(x, kind="stable")
+    d = np.diff(q[order])
+    assert (d >= 0).all() if scale > 0 else (d <= 0).all()
