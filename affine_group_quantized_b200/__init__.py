@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.qmv_last_error.argtypes = []
         L.qmv_abi_version.restype = I
         L.qmv_abi_version.argtypes = []
+        L.qmv_device_status.argtypes = [P, I, P]
+        L.qmv_device_status.restype = I
         L.affine_quantize.argtypes = [P, P, P, P, I, I, I, I, P]
         L.affine_dequantize.argtypes = [P, P, P, P, I, I, I, I, P]
         L.affine_quantize.restype = I
@@ -74,8 +76,8 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-EXPORTED = ("qmv", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
-            "qmv_last_error", "qmv_abi_version", "affine_quantize",
+EXPORTED = ("qmv", "qmv_noalloc", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
+            "qmv_last_error", "qmv_abi_version", "qmv_device_status", "affine_quantize",
             "affine_dequantize", "qmv_quant_last_error")
 
 
@@ -112,6 +114,15 @@ def last_error() -> str:
 
 def abi_version() -> int:
     return lib().qmv_abi_version()
+
+
+def device_status(reset=False, stream=None) -> int:
+    """The current device's kernel status word (0, or 2 if a bounded wait in
+    some kernel gave up since the last reset); synchronizes `stream`."""
+    out = ctypes.c_int(-1)
+    _check("qmv_device_status", lib().qmv_device_status(ctypes.byref(out), 1 if reset else 0,
+                                                        _stream(stream)))
+    return out.value
 
 
 def qmv(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):

@@ -16,6 +16,7 @@
 #include <cuda_fp16.h>
 
 #include "qmv.h"
+#include "qmv_decode.cuh"
 #include "qmv_mma.cuh"
 #include "qmv_stream.cuh"
 
@@ -79,10 +80,17 @@ int gcd_i(int a, int b) {
   return a;
 }
 
+// Status word of the GEMV kernels, one per device: a kernel ORs 2 into it
+// when one of its bounded waits gives up (that launch's results are then
+// undefined).  Read and cleared with qmv_device_status.
+static __device__ int g_device_status;
+
 // Per-device facts, queried once per device.
 struct DeviceInfo {
   int sms = 0;
   int smem_optin = 0;
+  int *status = nullptr;        // device address of g_device_status
+  cudaError_t status_err = cudaSuccess;
 };
 constexpr int kMaxDevices = 64;
 #ifndef QMV_MMA_MIN_ROWS
@@ -107,9 +115,16 @@ int device_info(DeviceInfo **out) {
     cudaError_t e2 = cudaDeviceGetAttribute(
         &g_dev[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e1 != cudaSuccess || e2 != cudaSuccess) g_dev[dev].sms = 0;
+    // the status word's device address, with this device current
+    void *a = nullptr;
+    g_dev[dev].status_err = cudaGetSymbolAddress(&a, g_device_status);
+    if (g_dev[dev].status_err == cudaSuccess) g_dev[dev].status = static_cast<int *>(a);
   });
   if (g_dev[dev].sms <= 0)
     return fail(QMV_ERR_CUDA, "cannot query device %d attributes", dev);
+  if (!g_dev[dev].status)
+    return fail(QMV_ERR_CUDA, "cudaGetSymbolAddress(status word): %s",
+                cudaGetErrorString(g_dev[dev].status_err));
   *out = &g_dev[dev];
   return rc;
 }
@@ -327,6 +342,135 @@ int launch(const Plan &pl, int bits, cudaStream_t stream) {
 void init_params(qmvk::StreamParams &p) { std::memset(&p, 0, sizeof p); }
 
 // ---------------------------------------------------------------------------
+// The decode kernel (qmv_decode.cuh): one activation row, 2- or 4-bit codes,
+// rows of a multiple of 2048 codes.  Other shapes take the streaming kernel.
+// ---------------------------------------------------------------------------
+
+// The decode kernel takes 2- and 4-bit codes, where the streaming kernel's
+// per-code work was the limit; for 3-, 5-, 6- and 8-bit codes the streaming
+// kernel measured as fast or faster.
+bool decode_path(int M, int K, int bits) {
+  return M == 1 && (bits == 2 || bits == 4) && K % 2048 == 0 && K <= 28672;
+}
+
+struct DecodePlan {
+  qmvk::DecodeParams p;
+  int grid = 0, threads = 0;
+  size_t smem = 0;
+};
+
+// Consumer warps: the most whole rows of warps (K / 2048 warps per row)
+// within kDecodeMaxWarps; slots of decode_rps<BITS>() rows per row phase; as many
+// slots as fit next to the partial sums, the span records, the activations
+// and the barriers.  Returns false when not even two slots fit (the caller
+// then takes the streaming kernel).
+bool make_decode_plan(DecodePlan &dp, int bits, int gs, bool silu, DeviceInfo *dev) {
+  qmvk::DecodeParams &p = dp.p;
+  const int K = p.K;
+  const int rps = qmvk::kDecodeRps;
+  const int rec_words = qmvk::kSpanRec;
+  p.WPR = K / 2048;
+  p.G = K / gs;
+  p.row_bytes = static_cast<uint32_t>(static_cast<long long>(K) * bits / 8);
+  const long long dig = static_cast<long long>(K / qmvk::kSpan) * rec_words * 4;
+  const long long xs = (silu ? 4LL : 2LL) * K;
+  // the most row phases whose ring still holds three slots (two if even one
+  // row phase does not)
+  int best_ph = 0, best_ns = 0;
+  for (int ph = qmvk::kDecodeMaxWarps / p.WPR; ph >= 1; --ph) {
+    const int SR = ph * rps;
+    const long long slot_w = static_cast<long long>(SR) * p.row_bytes;
+    const long long slot_s = static_cast<long long>(SR) * 2 * p.G;
+    const long long slot_bytes = (slot_w + 2 * slot_s + 127) / 128 * 128;
+    int ns = 0;
+    for (int k = 32; k >= 2; --k) {
+      const long long part = (static_cast<long long>(k) * 2 * SR * p.WPR * 4 + 15) / 16 * 16;
+      if (static_cast<long long>(k) * slot_bytes + part + dig + xs + 2LL * k * 8 <=
+          dev->smem_optin) {
+        ns = k;
+        break;
+      }
+    }
+    if (ns >= 3 || (ns >= 2 && ph == 1)) {
+      best_ph = ph;
+      best_ns = ns;
+      break;
+    }
+  }
+  if (best_ns < 2) return false;
+  p.PH = best_ph;
+  p.SR = p.PH * rps;
+  p.slot_w = static_cast<uint32_t>(p.SR) * p.row_bytes;
+  p.slot_s = static_cast<uint32_t>(p.SR) * 2u * static_cast<uint32_t>(p.G);
+  p.slot_bytes = (p.slot_w + 2 * p.slot_s + 127) / 128 * 128;
+  p.nslot = best_ns;
+  const long long part = (static_cast<long long>(p.nslot) * 2 * p.SR * p.WPR * 4 + 15) / 16 * 16;
+  p.part_off = static_cast<uint32_t>(static_cast<long long>(p.nslot) * p.slot_bytes);
+  p.dig_off = static_cast<uint32_t>(p.part_off + part);
+  p.x_off = static_cast<uint32_t>(p.dig_off + dig);
+  p.bar_off = static_cast<uint32_t>(p.x_off + xs);
+  dp.smem = static_cast<size_t>(p.bar_off) + 2u * p.nslot * 8;
+  long long grid = dev->sms;
+  if (p.total_rows < grid) grid = p.total_rows;
+  dp.grid = static_cast<int>(grid);
+  dp.threads = (p.WPR * p.PH + 1) * 32;
+  return true;
+}
+
+template <int BITS, int GS, bool SILU>
+int launch_decode_t(const DecodePlan &dp, cudaStream_t stream) {
+  auto kern = qmvk::qmv_decode_kernel<BITS, GS, SILU>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int granted[kMaxDevices] = {};
+  if (static_cast<int>(dp.smem) > granted[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(dp.smem));
+    if (e != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    granted[dev] = static_cast<int>(dp.smem);
+  }
+  const cudaError_t le = launch_pdl(kern, dp.grid, dp.threads, static_cast<int>(dp.smem),
+                                    stream, dp.p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(le));
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(QMV_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+template <int BITS, bool SILU>
+int launch_decode_b(const DecodePlan &dp, int gs, cudaStream_t stream) {
+  switch (gs) {
+    case 32: return launch_decode_t<BITS, 32, SILU>(dp, stream);
+    case 64: return launch_decode_t<BITS, 64, SILU>(dp, stream);
+    case 128: return launch_decode_t<BITS, 128, SILU>(dp, stream);
+    default: return fail(QMV_ERR_UNSUPPORTED, "group_size=%d", gs);
+  }
+}
+
+template <bool SILU>
+int launch_decode(const DecodePlan &dp, int bits, int gs, cudaStream_t stream) {
+  switch (bits) {
+    case 2: return launch_decode_b<2, SILU>(dp, gs, stream);
+    case 4: return launch_decode_b<4, SILU>(dp, gs, stream);
+    default: return fail(QMV_ERR_UNSUPPORTED, "bits=%d on the decode kernel", bits);
+  }
+}
+
+// Fills the matrix-independent fields of a decode plan.
+void init_decode(DecodePlan &dp, const void *x, int N, int K, int nmat, const DeviceInfo *dev) {
+  std::memset(&dp.p, 0, sizeof dp.p);
+  dp.p.err = dev->status;
+  dp.p.x = static_cast<const uint16_t *>(x);
+  dp.p.N = N;
+  dp.p.K = K;
+  dp.p.total_rows = static_cast<long long>(nmat) * N;
+}
+
+// ---------------------------------------------------------------------------
 // Batched rows on the tensor cores (qmv_mma.cuh): up to 16 activation rows
 // share one read of the weights.  2-, 4- and 8-bit codes; K a multiple of
 // one stage row (1024 / bits codes); group sizes 32, 64, 128.
@@ -386,7 +530,7 @@ struct MmaScratch {
 MmaScratch g_mma_scratch[kMaxDevices];
 std::mutex g_mma_scratch_mu;
 
-int mma_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
+int mma_scratch(int dev_id, int sms, int ntiles, cudaStream_t stream, MmaScratch **out) {
   std::lock_guard<std::mutex> lock(g_mma_scratch_mu);
   MmaScratch &s = g_mma_scratch[dev_id];
   if (!s.part) {
@@ -398,9 +542,14 @@ int mma_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
     int n = s.cnt_len ? s.cnt_len : 1024;
     while (n < ntiles) n *= 2;
     int *c = nullptr;
-    if (cudaMalloc(&c, static_cast<size_t>(n) * 4) != cudaSuccess ||
-        cudaMemset(c, 0, static_cast<size_t>(n) * 4) != cudaSuccess)
+    // zeroed on the caller's stream, so the launch that follows on that
+    // stream sees the zeros whatever kind of stream it is
+    if (cudaMalloc(&c, static_cast<size_t>(n) * 4) != cudaSuccess)
       return fail(QMV_ERR_CUDA, "tensor-core path: cannot allocate the tile counters");
+    if (cudaMemsetAsync(c, 0, static_cast<size_t>(n) * 4, stream) != cudaSuccess) {
+      cudaFree(c);
+      return fail(QMV_ERR_CUDA, "tensor-core path: cannot clear the tile counters");
+    }
     if (s.cnt) cudaFree(s.cnt);  // waits for the launches that use it
     s.cnt = c;
     s.cnt_len = n;
@@ -419,6 +568,7 @@ constexpr size_t kStaticPartBytes =
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticPartBytes +
                                                                  kStaticTiles * 4];
 MmaScratch g_static_view[kMaxDevices];
+cudaError_t g_static_err[kMaxDevices];
 std::once_flag g_static_once[kMaxDevices];
 
 int static_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
@@ -426,10 +576,10 @@ int static_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
     return fail(QMV_ERR_UNSUPPORTED,
                 "qmv_noalloc: %d SMs / %d row tiles exceed the fixed scratch (%d / %d)", sms,
                 ntiles, kStaticCtas, kStaticTiles);
-  cudaError_t e = cudaSuccess;
   std::call_once(g_static_once[dev_id], [&] {
     void *a = nullptr;
-    e = cudaGetSymbolAddress(&a, g_static_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&a, g_static_scratch);
+    g_static_err[dev_id] = e;
     if (e == cudaSuccess) {
       g_static_view[dev_id].part = static_cast<float *>(a);
       g_static_view[dev_id].cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(a) +
@@ -438,7 +588,8 @@ int static_scratch(int dev_id, int sms, int ntiles, MmaScratch **out) {
     }
   });
   if (!g_static_view[dev_id].part)
-    return fail(QMV_ERR_CUDA, "qmv_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    return fail(QMV_ERR_CUDA, "qmv_noalloc: cudaGetSymbolAddress: %s",
+                cudaGetErrorString(g_static_err[dev_id]));
   *out = &g_static_view[dev_id];
   return 0;
 }
@@ -538,10 +689,11 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   MmaScratch *sc = nullptr;
   int rc;
   if ((rc = fixed_scratch ? static_scratch(d, dev->sms, mp.ntiles, &sc)
-                         : mma_scratch(d, dev->sms, mp.ntiles, &sc)))
+                         : mma_scratch(d, dev->sms, mp.ntiles, stream, &sc)))
     return rc;
   mp.part = sc->part;
   mp.cnt = sc->cnt;
+  mp.err = dev->status;
   switch (bits) {
     case 2: return launch_mma_b<2>(mp, gs, grid, dev, stream);
     case 4: return launch_mma_b<4>(mp, gs, grid, dev, stream);
@@ -566,6 +718,16 @@ int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *sca
   if (mma_path(M, K, bits, group_size))
     return launch_mma(x, w, scales, biases, y, M, N, K, bits, group_size, dev,
                       static_cast<cudaStream_t>(stream), fixed_scratch);
+  if (decode_path(M, K, bits)) {
+    DecodePlan dp;
+    init_decode(dp, x, N, K, 1, dev);
+    dp.p.w[0] = reinterpret_cast<const uint8_t *>(w);
+    dp.p.s[0] = static_cast<const uint16_t *>(scales);
+    dp.p.b[0] = static_cast<const uint16_t *>(biases);
+    dp.p.y[0] = static_cast<uint16_t *>(y);
+    if (make_decode_plan(dp, bits, group_size, false, dev))
+      return launch_decode<false>(dp, bits, group_size, static_cast<cudaStream_t>(stream));
+  }
   Plan pl;
   init_params(pl.p);
   qmvk::StreamParams &p = pl.p;
@@ -580,6 +742,7 @@ int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *sca
   p.K = K;
   p.nmat = 1;
   p.total_rows = N;
+  p.err = dev->status;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -589,6 +752,19 @@ int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *sca
 extern "C" {
 
 int qmv_abi_version(void) { return 1; }
+
+int qmv_device_status(int *out, int reset, void *stream) {
+  if (!out) return fail(QMV_ERR_NULL, "qmv_device_status: out is NULL");
+  DeviceInfo *dev;
+  int rc;
+  if ((rc = device_info(&dev))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(out, dev->status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && reset) e = cudaMemsetAsync(dev->status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return fail(QMV_ERR_CUDA, "qmv_device_status: %s", cudaGetErrorString(e));
+  return ok();
+}
 
 const char *qmv_last_error(void) { return g_last_error.c_str(); }
 
@@ -622,6 +798,20 @@ int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
       return fail(QMV_ERR_ALIGN, "qmv_gate_up: buffers must be 16-byte aligned");
   DeviceInfo *dev;
   if ((rc = device_info(&dev))) return rc;
+  if (decode_path(M, K, bits)) {
+    DecodePlan dp;
+    init_decode(dp, x, N, K, 2, dev);
+    dp.p.w[0] = reinterpret_cast<const uint8_t *>(w_gate);
+    dp.p.s[0] = static_cast<const uint16_t *>(s_gate);
+    dp.p.b[0] = static_cast<const uint16_t *>(b_gate);
+    dp.p.y[0] = static_cast<uint16_t *>(y_gate);
+    dp.p.w[1] = reinterpret_cast<const uint8_t *>(w_up);
+    dp.p.s[1] = static_cast<const uint16_t *>(s_up);
+    dp.p.b[1] = static_cast<const uint16_t *>(b_up);
+    dp.p.y[1] = static_cast<uint16_t *>(y_up);
+    if (make_decode_plan(dp, bits, group_size, false, dev))
+      return launch_decode<false>(dp, bits, group_size, static_cast<cudaStream_t>(stream));
+  }
   Plan pl;
   init_params(pl.p);
   qmvk::StreamParams &p = pl.p;
@@ -640,6 +830,7 @@ int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,
   p.K = K;
   p.nmat = 2;
   p.total_rows = N;
+  p.err = dev->status;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -663,6 +854,18 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
     return fail(QMV_ERR_ALIGN, "qmv_silu_gate_resid: x_resid must be 2-byte aligned");
   DeviceInfo *dev;
   if ((rc = device_info(&dev))) return rc;
+  if (decode_path(M, K, bits)) {
+    DecodePlan dp;
+    init_decode(dp, gate, N, K, 1, dev);
+    dp.p.up = static_cast<const uint16_t *>(up);
+    dp.p.resid = static_cast<const uint16_t *>(x_resid);
+    dp.p.w[0] = reinterpret_cast<const uint8_t *>(w);
+    dp.p.s[0] = static_cast<const uint16_t *>(scales);
+    dp.p.b[0] = static_cast<const uint16_t *>(biases);
+    dp.p.y[0] = static_cast<uint16_t *>(y);
+    if (make_decode_plan(dp, bits, group_size, true, dev))
+      return launch_decode<true>(dp, bits, group_size, static_cast<cudaStream_t>(stream));
+  }
   Plan pl;
   init_params(pl.p);
   qmvk::StreamParams &p = pl.p;
@@ -679,6 +882,7 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
   p.K = K;
   p.nmat = 1;
   p.total_rows = N;
+  p.err = dev->status;
   if ((rc = make_plan(pl, bits, group_size, M, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
@@ -737,6 +941,9 @@ int gather_qmv(const void *x, const uint32_t *w, const void *scales,
   p.num_x_rows = num_x_rows;
   p.num_experts = num_experts;
   p.total_rows = static_cast<long long>(num_experts) * N;
+  // a bounded wait that gives up is reported in the caller's status word
+  // when there is one
+  p.err = d_status ? d_status : dev->status;
   const int mr = num_pairs >= num_experts ? 2 : 1;
   if ((rc = make_plan(pl, bits, group_size, mr, dev))) return rc;
   return launch(pl, bits, static_cast<cudaStream_t>(stream));

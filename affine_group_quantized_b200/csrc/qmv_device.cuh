@@ -72,6 +72,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   return false;
 }
 
+// Bounded wait that lets the waiting thread sleep: each try_wait may
+// suspend the thread for up to 10 us, or until the phase completes.  The
+// bound (2^16 rounds, well under a second) only ends a broken launch.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 16); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(10000u)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 // 1-D bulk copy global -> shared, completing `bytes` on `bar`.  Both
 // addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src,
@@ -102,6 +122,70 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
 }
 __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Warp reductions
+// ---------------------------------------------------------------------------
+
+// c ? a : b on values, kept a register select (a select between two array
+// elements may otherwise become an indexed load from local memory).
+__device__ __forceinline__ float select_f32(bool c, float a, float b) {
+  float r;
+  asm("{\n.reg .pred q;\nsetp.ne.u32 q, %3, 0;\nselp.f32 %0, %1, %2, q;\n}\n"
+      : "=f"(r)
+      : "f"(a), "f"(b), "r"(static_cast<uint32_t>(c)));
+  return r;
+}
+
+// Transposed butterfly over the 32 lanes of a warp: NV partial sums per lane
+// in; afterwards lane l holds the full sum of value l / (32 / NV) in vals[0].
+template <int NV>
+__device__ __forceinline__ void transpose_reduce(float (&vals)[NV], int lane) {
+  static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "NV");
+  const unsigned full = 0xffffffffu;
+#pragma unroll
+  for (int off = 16, n = NV; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < n / 2; ++i) {
+        const float lo = vals[i], hi = vals[i + n / 2];
+        const float send = select_f32(upper, lo, hi);
+        const float keep = select_f32(upper, hi, lo);
+        vals[i] = keep + __shfl_xor_sync(full, send, off);
+      }
+      n >>= 1;
+    } else {
+      vals[0] += __shfl_xor_sync(full, vals[0], off);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -302,26 +302,6 @@ struct RingPos {
   }
 };
 
-// Bounded wait that lets the waiting thread sleep: each try_wait may
-// suspend the thread for up to 10 us, or until the phase completes.  The
-// bound (2^16 rounds, well under a second) only ends a broken launch.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 16); ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n"
-        ".reg .pred p;\n"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        "selp.u32 %0, 1, 0, p;\n"
-        "}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(10000u)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
-}
-
 // ---------------------------------------------------------------------------
 // Dequant: one 32-bit word of codes -> fp16 w_hat, as half2 pairs, in the
 // word's permuted k order (see the top of the file).

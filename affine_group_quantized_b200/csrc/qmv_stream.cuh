@@ -323,32 +323,6 @@ __device__ __forceinline__ long long abs_row(const StreamParams &p, int arr,
                                : static_cast<long long>(row);
 }
 
-// ---------------------------------------------------------------------------
-// Shared-memory helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(a));
-  return v;
-}
-
 // One unit (4*BITS bytes, starting at a multiple of 4*BITS) from shared
 // memory with the widest aligned loads.
 template <int BITS>
@@ -560,40 +534,6 @@ __device__ __forceinline__ void epilogue_loop(const StreamParams &p,
 // Consumers
 // ---------------------------------------------------------------------------
 
-// c ? a : b on values, kept a register select (a select between two array
-// elements may otherwise become an indexed load from local memory).
-__device__ __forceinline__ float select_f32(bool c, float a, float b) {
-  float r;
-  asm("{\n.reg .pred q;\nsetp.ne.u32 q, %3, 0;\nselp.f32 %0, %1, %2, q;\n}\n"
-      : "=f"(r)
-      : "f"(a), "f"(b), "r"(static_cast<uint32_t>(c)));
-  return r;
-}
-
-// Transposed butterfly over the 32 lanes of a warp: NV partial sums per lane
-// in; afterwards lane l holds the full sum of value l / (32 / NV) in vals[0].
-template <int NV>
-__device__ __forceinline__ void transpose_reduce(float (&vals)[NV], int lane) {
-  static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "NV");
-  const unsigned full = 0xffffffffu;
-#pragma unroll
-  for (int off = 16, n = NV; off >= 1; off >>= 1) {
-    if (n > 1) {
-      const bool upper = (lane & off) != 0;
-#pragma unroll
-      for (int i = 0; i < n / 2; ++i) {
-        const float lo = vals[i], hi = vals[i + n / 2];
-        const float send = select_f32(upper, lo, hi);
-        const float keep = select_f32(upper, hi, lo);
-        vals[i] = keep + __shfl_xor_sync(full, send, off);
-      }
-      n >>= 1;
-    } else {
-      vals[0] += __shfl_xor_sync(full, vals[0], off);
-    }
-  }
-}
-
 // The raw bf16 words of one unit's activations for one activation row (and,
 // in MODE_SILU, of `up`).
 struct UnitRaw {
@@ -750,7 +690,7 @@ template <int BITS, int MR, int NSL, bool SILU, bool BIG = false>
 __global__ void __launch_bounds__(BIG ? 512 : 576, 1)
     qmv_stream_kernel(const StreamParams p) {
   constexpr int RPT = rows_per_thread<BITS, MR, NSL, BIG>();
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x;
   const int Tc = p.Upad * p.PH / NSL;  // consumer threads
   const uint32_t slot_bytes = p.w_slot + 2 * p.s_slot;

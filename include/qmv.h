@@ -30,19 +30,21 @@
  * Conventions
  * ---------------------------------------------------------------------------
  * Pointers: every buffer pointer is a DEVICE pointer owned by the caller and
- * must be 16-byte aligned.  The library never frees or retains them and does
- * not allocate device memory.
+ * must be 16-byte aligned.  The library never frees or retains them.  It
+ * allocates device memory in one place only: qmv's tensor-core path (several
+ * activation rows) allocates its split-tile scratch on the first such call on
+ * a device, and grows it when a call needs more; qmv_noalloc takes the same
+ * operation without any allocation, and no other entry point allocates.
  * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  * Every call only enqueues work on that stream and returns; results are
- * ready when the stream is synchronized.  Each successful call enqueues
- * exactly one kernel.
- * Errors: every argument is checked on the host before anything is
- * enqueued; on a bad argument nothing touches the device and the call
- * returns a nonzero qmv_status.  qmv_last_error() then describes the failure
- * (thread-local; valid until the next call on the same thread).  There is no
- * silent fallback: a combination without a kernel returns
- * QMV_ERR_UNSUPPORTED (the pages' QuantWeights trait makes its fused
- * operations return an error rather than take a slow path).
+ * ready when the stream is synchronized.  Each successful call enqueues one
+ * kernel (qmv's tensor-core path also enqueues a clear of new scratch, on
+ * the same stream, when it allocates).
+ * Bounded waits: every wait inside the kernels gives up after a bound (a few
+ * hundred milliseconds); a kernel whose wait gave up ORs 2 into a status
+ * word -- gather_qmv's d_status when given, else the library's per-device
+ * word that qmv_device_status reads -- and that launch's results are
+ * undefined.  In a correct launch no wait comes near the bound.
  */
 #ifndef LIBQMV_QMV_H
 #define LIBQMV_QMV_H
@@ -159,7 +161,8 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
  *                (bit-identical), whatever the order of the pairs.
  *   d_status     device int or NULL.  If any index is out of range the
  *                kernel ORs 1 into *d_status and leaves that pair's output
- *                row unwritten; valid pairs are still computed.  The caller
+ *                row unwritten; valid pairs are still computed.  A bounded
+ *                wait that gave up ORs 2 (see Conventions).  The caller
  *                zeroes *d_status before the call.
  * The kernel reads every expert that some pair uses once per call, whether or
  * not the indices are sorted.  num_pairs may be 0 (nothing is enqueued).
@@ -230,6 +233,19 @@ const char *qmv_last_error(void);
 
 /* ABI version of this header (incremented on incompatible change). */
 int qmv_abi_version(void);
+
+/*
+ * qmv_device_status -- read the current device's status word of the GEMV
+ * kernels (no counterpart on the pages; part of this library's bounded-wait
+ * error reporting, see Conventions).
+ *   out     HOST int, written with the word: 0, or 2 if some kernel's
+ *           bounded wait gave up since the last reset
+ *   reset   nonzero: clear the word afterwards (enqueued on `stream`)
+ *   stream  the word is read after the work already enqueued on `stream`;
+ *           the call synchronizes that stream
+ * Returns QMV_ERR_NULL for a NULL out, QMV_ERR_CUDA if a CUDA call fails.
+ */
+int qmv_device_status(int *out, int reset, void *stream);
 
 #ifdef __cplusplus
 }

@@ -114,3 +114,75 @@ def test_two_digit_fixed_point_would_fail_the_outlier_unit():
     x, codes, w, s, b, N, K, bits, gs = _outlier_case()
     y_ref, a_ref = oracle.qmv(x, w, s, b, 1, N, K, bits, gs)
     assert _ratio(_model(x, codes, s, b, gs, ndigits=2), y_ref, a_ref) > 1.0
+
+
+# ---------------------------------------------------------------------------
+# The decode kernel (one activation row, 2/4-bit codes, rows of a multiple of
+# 2048 codes): each thread owns a 64-code span; one power of two per span
+# (so the fixed point covers 64 activations); per group part of the span
+# (one part, or two for group size 32) the digit sums are combined exactly
+# (S0 + 256 S1 + 65536 S2 as two fp32 additions of exact terms), multiplied
+# by the scale and added up over the parts; the bias term uses the part's
+# fp32 activation sum; the span result is sr * 2^-s + bs; the spans of a row
+# are added in fp32.
+# ---------------------------------------------------------------------------
+
+def _model_span(x_bits, codes, s_bits, b_bits, gs, ndigits=3, span=64):
+    x = synth.bits_to_float(x_bits).astype(np.float32)[0]
+    s = synth.bits_to_float(s_bits).astype(np.float32)
+    b = synth.bits_to_float(b_bits).astype(np.float32)
+    N, K = codes.shape
+    top = 8 * ndigits - 2
+    parts = 2 if gs == 32 else 1
+    plen = span // parts
+    y = np.zeros(N, np.float32)
+    for t in range(K // span):
+        xs = x[span * t:span * t + span]
+        mx = float(np.max(np.abs(xs)))
+        eb = int(np.frexp(np.float32(mx))[1]) + 126 if mx > 0 else 0
+        sh = int(np.clip(top + 126 - eb, -126, 126))
+        X = np.rint(xs.astype(np.float64) * 2.0 ** sh).astype(np.int64)
+        assert np.all(np.abs(X) <= 2 ** top)
+        d, rest = [], X.copy()
+        for i in range(ndigits - 1):
+            d.append(rest & 0xFF)
+            rest = rest >> 8
+        d.append(rest)
+        sr = np.zeros(N, np.float32)
+        bs = np.zeros(N, np.float32)
+        for h in range(parts):
+            lo, hi = span * t + plen * h, span * t + plen * (h + 1)
+            q = codes[:, lo:hi].astype(np.int64)
+            sums = [q @ di[plen * h:plen * (h + 1)] for di in d]   # exact integers
+            r = (sums[0] * 1.0).astype(np.float32)
+            for i in range(1, ndigits):
+                r = f32(r.astype(np.float64) + sums[i].astype(np.float64) * 256.0 ** i)
+            vs = f32(0.0)
+            for v in x[lo:hi]:
+                vs = f32(vs + v)
+            g = lo // gs
+            sr = f32(s[:, g].astype(np.float64) * r.astype(np.float64) + sr.astype(np.float64))
+            bs = f32(b[:, g].astype(np.float64) * float(vs) + bs.astype(np.float64))
+        part = f32(sr.astype(np.float64) * 2.0 ** -sh + bs.astype(np.float64))
+        y = f32(y + part)
+    return _bf16_round(y.astype(np.float64))[None, :]
+
+
+@pytest.mark.parametrize("bits, gs", [(4, 64), (2, 32), (4, 128), (2, 64)])
+def test_decode_span_roundings_meet_the_bound(bits, gs):
+    N, K = 32, 2048
+    x, codes, w, s, b = _inputs(N, K, bits, gs, seed=600 + bits + gs)
+    y_ref, a_ref = oracle.qmv(x, w, s, b, 1, N, K, bits, gs)
+    assert _ratio(_model_span(x, codes, s, b, gs), y_ref, a_ref) <= 1.0
+
+
+def test_decode_span_outlier_meets_the_bound():
+    x, codes, w, s, b, N, K, bits, gs = _outlier_case()
+    y_ref, a_ref = oracle.qmv(x, w, s, b, 1, N, K, bits, gs)
+    assert _ratio(_model_span(x, codes, s, b, gs), y_ref, a_ref) <= 1.0
+
+
+def test_decode_span_two_digits_would_fail_the_outlier():
+    x, codes, w, s, b, N, K, bits, gs = _outlier_case()
+    y_ref, a_ref = oracle.qmv(x, w, s, b, 1, N, K, bits, gs)
+    assert _ratio(_model_span(x, codes, s, b, gs, ndigits=2), y_ref, a_ref) > 1.0

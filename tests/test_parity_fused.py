@@ -32,9 +32,10 @@ def _silu(g, u, r, w, s, b, M, N, K, bits, gs):
     return host_bits(Y)
 
 
-@pytest.mark.parametrize("bits", [4, 8, 3])
-def test_gate_up_small(bits):
-    gs, M, N, K = 64, 1, 333, 1024
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("M", [1, 2])
+def test_gate_up_small(bits, M):
+    gs, N, K = 64, 333, 1024
     x, wg, sg, bg = synth.qmv_inputs(M, N, K, bits, gs, seed=11)
     _, wu, su, bu = synth.qmv_inputs(M, N, K, bits, gs, seed=12)
     yg, yu = _gate_up(x, wg, sg, bg, wu, su, bu, M, N, K, bits, gs)
@@ -68,7 +69,7 @@ def test_ffn_int8_full_size():
     check(yd[:, rows2], rd, ad, "ffn down (silu-gate-resid)")
 
 
-@pytest.mark.parametrize("bits", [2, 4, 5, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("with_resid", [True, False])
 def test_silu_gate_resid_small(bits, with_resid):
     gs, M, N, K = 32, 2, 77, 2048
@@ -126,12 +127,13 @@ def test_gather_moe_workload_sorted_and_unsorted():
         check(y_u[p:p + 1], y_ref[p:p + 1], a_ref[p:p + 1], f"gather pair {p}")
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
-def test_gather_small_routing(bits):
-    E, N, K, gs, T = 9, 70, 512, 64, 6
-    w, s, b = _moe_inputs(E, N, K, bits, gs, seed=bits)
+@pytest.mark.parametrize("bits, gs", [(2, 64), (3, 64), (4, 64), (5, 64), (6, 64), (8, 64),
+                                      (4, 128), (5, 128), (3, 32)])
+def test_gather_small_routing(bits, gs):
+    E, N, K, T = 9, 70, 512, 6
+    w, s, b = _moe_inputs(E, N, K, bits, gs, seed=bits + gs)
     x = synth.normal_bf16((T, K), seed=bits + 1)
-    rng = np.random.default_rng(bits)
+    rng = np.random.default_rng(bits + gs)
     P = 23
     lhs = rng.integers(0, T, size=P).astype(np.uint32)
     rhs = rng.integers(0, E, size=P).astype(np.uint32)
@@ -139,7 +141,7 @@ def test_gather_small_routing(bits):
     y, st = _gather(x, w, s, b, lhs, rhs, P, T, E, N, K, bits, gs, False)
     assert st == 0
     y_ref, a_ref, valid = oracle.gather(x, w, s, b, lhs, rhs, P, T, E, N, K, bits, gs)
-    check(y, y_ref, a_ref, f"gather bits={bits}")
+    check(y, y_ref, a_ref, f"gather bits={bits} gs={gs}")
 
 
 def test_gather_identity_lhs_and_bad_indices():
