@@ -83,12 +83,15 @@ def workload(name):
         _, wu, su, bu = synth.qmv_inputs(M, N, K, bits, gs, seed=3001, **kw)
         _, wd, sd, bd = synth.qmv_inputs(M, K, N, bits, gs, seed=3002, **kw)
         resid = synth.normal_bf16((M, K), seed=3003)
+        # input of the down projection: gate and up activations (synthetic)
+        gate = synth.normal_bf16((M, N), seed=3004)
+        up = synth.normal_bf16((M, N), seed=3005)
         gu_bytes = 2 * (N * K + 4 * N * (K // gs)) + 2 * K + 2 * 2 * N
         dn_bytes = K * N + 4 * K * (N // gs) + 2 * 2 * N + 2 * K + 2 * K
         L.append(Launch("gate_up_int8", "gate_up", gu_bytes, M=M, N=N, K=K, bits=bits,
                         gs=gs, x=x, wg=wg, sg=sg, bg=bg, wu=wu, su=su, bu=bu))
         L.append(Launch("silu_down_int8", "silu", dn_bytes, M=M, N=K, K=N, bits=bits,
-                        gs=gs, w=wd, s=sd, b=bd, resid=resid))
+                        gs=gs, w=wd, s=sd, b=bd, resid=resid, gate=gate, up=up))
         cfg = {"workload": "fused FFN decode int8", "K": K, "N": N, "group_size": gs,
                "bits": bits}
     elif name == "batched":
@@ -144,58 +147,129 @@ def _dev(a, torch):
     return torch.from_numpy(a.view(np.int32)).cuda()
 
 
-class DeviceLaunch:
-    """Device buffers of one Launch, with `copies` rotating weight copies."""
+# Per launch kind: the arrays rotated across weight copies, the per-step
+# inputs (copied from the host in the end-to-end timing) and the outputs.
+_WEIGHTS = {"qmv": ("w", "s", "b"), "gate_up": ("wg", "sg", "bg", "wu", "su", "bu"),
+            "silu": ("w", "s", "b"), "gather": ("w", "s", "b"),
+            "quantize": ("w",), "dequantize": ("w", "s", "b")}
+_INPUTS = {"qmv": ("x",), "gate_up": ("x",), "silu": ("gate", "up", "resid"),
+           "gather": ("x", "lhs", "rhs"), "quantize": ("w",), "dequantize": ()}
 
-    def __init__(self, l, copies, torch):
+
+def _outputs(l):
+    """(name, shape, numpy dtype) of the arrays a launch writes."""
+    if l.kind == "qmv":
+        return [("y", (l.M, l.N), np.uint16)]
+    if l.kind == "gate_up":
+        return [("yg", (l.M, l.N), np.uint16), ("yu", (l.M, l.N), np.uint16)]
+    if l.kind == "silu":
+        return [("y", (l.M, l.N), np.uint16)]
+    if l.kind == "gather":
+        return [("y", (l.P, l.N), np.uint16)]
+    if l.kind == "quantize":
+        G = l.K // l.gs
+        return [("q", (l.N, l.K * l.bits // 32), np.uint32), ("s", (l.N, G), np.uint16),
+                ("b", (l.N, G), np.uint16)]
+    return [("y", (l.N, l.K), np.uint16)]   # dequantize
+
+
+class _Packed:
+    """One device buffer (and one pinned host buffer) holding several arrays
+    back to back at 16-byte aligned offsets, each reachable as a typed view:
+    a step's host copies are then one transfer each way."""
+
+    def __init__(self, specs, torch):
+        self.offsets, off = [], 0
+        for _, shape, dt in specs:
+            nb = int(np.prod(shape)) * np.dtype(dt).itemsize
+            self.offsets.append((off, nb, shape, dt))
+            off += (nb + 15) // 16 * 16
+        self.nbytes = max(off, 16)
+        self.dev = torch.empty(self.nbytes, dtype=torch.uint8, device="cuda")
+        self.host = torch.empty(self.nbytes, dtype=torch.uint8).pin_memory()
+        self.names = [n for n, _, _ in specs]
+        self.torch = torch
+
+    def view(self, i, buf=None):
+        torch = self.torch
+        off, nb, shape, dt = self.offsets[i]
+        t = (self.dev if buf is None else buf)[off:off + nb]
+        td = {np.uint16: torch.bfloat16, np.uint32: torch.int32, np.int32: torch.int32}[dt]
+        return t.view(td).view(shape)
+
+    def fill_host(self, arrays):
+        h = self.host.numpy()
+        for (off, nb, _, _), a in zip(self.offsets, arrays):
+            h[off:off + nb] = np.frombuffer(np.ascontiguousarray(a).tobytes(), np.uint8)
+
+
+class DeviceWorkload:
+    """Device buffers of a workload's launches.  Weights rotate over
+    `copies[i]` copies per launch i; each launch's per-step inputs and its
+    outputs are views into one packed input and one packed output buffer."""
+
+    def __init__(self, launches, copies, torch):
         import affine_group_quantized_b200 as agq
-        self.l, self.agq, self.torch = l, agq, torch
-        d = lambda a: _dev(a, torch)  # noqa: E731
-        self.copies = []
-        for _ in range(copies):
-            if l.kind == "qmv":
-                self.copies.append(dict(w=d(l.w), s=d(l.s), b=d(l.b)))
-            elif l.kind == "gate_up":
-                self.copies.append(dict(wg=d(l.wg), sg=d(l.sg), bg=d(l.bg),
-                                        wu=d(l.wu), su=d(l.su), bu=d(l.bu)))
-            elif l.kind == "silu":
-                self.copies.append(dict(w=d(l.w), s=d(l.s), b=d(l.b)))
-            elif l.kind == "gather":
-                self.copies.append(dict(w=d(l.w), s=d(l.s), b=d(l.b)))
-        bf = torch.bfloat16
-        if l.kind == "qmv":
-            self.x = d(l.x)
-            self.y = torch.empty((l.M, l.N), dtype=bf, device="cuda")
-        elif l.kind == "gate_up":
-            self.x = d(l.x)
-            self.yg = torch.empty((l.M, l.N), dtype=bf, device="cuda")
-            self.yu = torch.empty((l.M, l.N), dtype=bf, device="cuda")
-            self.y = self.yg
-        elif l.kind == "silu":
-            # input of the down projection: gate/up activations (synthetic)
-            self.gate = d(synth.normal_bf16((l.M, l.K), seed=3004))
-            self.up = d(synth.normal_bf16((l.M, l.K), seed=3005))
-            self.x = self.gate
-            self.resid = d(l.resid)
-            self.y = torch.empty((l.M, l.N), dtype=bf, device="cuda")
-        elif l.kind == "gather":
-            self.x = d(l.x)
-            self.lhs, self.rhs = d(l.lhs), d(l.rhs)
-            self.y = torch.empty((l.P, l.N), dtype=bf, device="cuda")
+        self.agq, self.torch, self.launches = agq, torch, launches
+        self.weights = []
+        for l, c in zip(launches, copies):
+            self.weights.append([{k: _dev(getattr(l, k), torch) for k in _WEIGHTS[l.kind]}
+                                 for _ in range(c)])
+        in_specs, out_specs, self.in_idx, self.out_idx = [], [], [], []
+        for l in launches:
+            idx = {}
+            for k in _INPUTS[l.kind]:
+                a = np.ascontiguousarray(getattr(l, k))
+                idx[k] = len(in_specs)
+                in_specs.append((k, a.shape, a.dtype.type))
+            self.in_idx.append(idx)
+            idx = {}
+            for k, shape, dt in _outputs(l):
+                idx[k] = len(out_specs)
+                out_specs.append((k, shape, dt))
+            self.out_idx.append(idx)
+        self.inp = _Packed(in_specs, torch)
+        self.out = _Packed(out_specs, torch)
+        arrays = [np.ascontiguousarray(getattr(l, k)) for l in launches for k in _INPUTS[l.kind]]
+        self.inp.fill_host(arrays)
+        self.inp.dev.copy_(self.inp.host)
+        self.h2d_bytes = sum(int(np.prod(s)) * np.dtype(d).itemsize for _, s, d in in_specs)
+        self.d2h_bytes = sum(int(np.prod(s)) * np.dtype(d).itemsize for _, s, d in out_specs)
 
-    def __call__(self, k):
-        l, c, agq = self.l, self.copies[k % len(self.copies)], self.agq
+    def run(self, i, k, e2e=False):
+        """Launch i with weight copy k (modulo its copies); end to end, the
+        quantizer reads the matrix just copied in from the host."""
+        l, agq = self.launches[i], self.agq
+        c = self.weights[i][k % len(self.weights[i])]
+        I = {n: self.inp.view(j) for n, j in self.in_idx[i].items()}
+        O = {n: self.out.view(j) for n, j in self.out_idx[i].items()}
         if l.kind == "qmv":
-            agq.qmv(self.x, c["w"], c["s"], c["b"], self.y, l.M, l.N, l.K, l.bits, l.gs)
+            agq.qmv(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.N, l.K, l.bits, l.gs)
         elif l.kind == "gate_up":
-            agq.qmv_gate_up(self.x, c["wg"], c["sg"], c["bg"], c["wu"], c["su"], c["bu"],
-                            self.yg, self.yu, l.M, l.N, l.K, l.bits, l.gs)
+            agq.qmv_gate_up(I["x"], c["wg"], c["sg"], c["bg"], c["wu"], c["su"], c["bu"],
+                            O["yg"], O["yu"], l.M, l.N, l.K, l.bits, l.gs)
         elif l.kind == "silu":
-            agq.qmv_silu_gate_resid(self.gate, self.up, self.resid, c["w"], c["s"], c["b"],
-                                    self.y, l.M, l.N, l.K, l.bits, l.gs)
+            agq.qmv_silu_gate_resid(I["gate"], I["up"], I["resid"], c["w"], c["s"], c["b"],
+                                    O["y"], l.M, l.N, l.K, l.bits, l.gs)
         elif l.kind == "gather":
-            agq.gather_qmv(self.x, c["w"], c["s"], c["b"], self.lhs, self.rhs, self.y,
+            agq.gather_qmv(I["x"], c["w"], c["s"], c["b"], I["lhs"], I["rhs"], O["y"],
                            l.P, l.T, l.E, l.N, l.K, l.bits, l.gs, sorted_indices=l.sorted)
+        elif l.kind == "quantize":
+            src = I["w"] if e2e else c["w"]
+            agq.affine_quantize(src, O["q"], O["s"], O["b"], l.N, l.K, l.bits, l.gs)
+        else:
+            agq.affine_dequantize(c["w"], c["s"], c["b"], O["y"], l.N, l.K, l.bits, l.gs)
+
+    def step(self, k, e2e=False):
+        for i in range(len(self.launches)):
+            self.run(i, k, e2e)
+
+    def e2e_step(self, k):
+        """One step as a user runs it: inputs in from pinned host memory, the
+        launches, the outputs back to pinned host memory."""
+        self.inp.dev.copy_(self.inp.host, non_blocking=True)
+        self.step(k, e2e=True)
+        self.out.host.copy_(self.out.dev, non_blocking=True)
 
 
 class ClockSampler:
@@ -260,7 +334,8 @@ class ClockSampler:
 # The sources the GEMV kernels and their launch plans are built from: the
 # recorded DRAM traffic is valid while these are unchanged.  (The producer
 # side of the format, qmv_quant.cu, has kernels of its own.)
-GEMV_SOURCES = ("qmv_api.cu", "qmv_device.cuh", "qmv_mma.cuh", "qmv_stream.cuh")
+GEMV_SOURCES = ("qmv_api.cu", "qmv_decode.cuh", "qmv_device.cuh", "qmv_mma.cuh",
+                "qmv_stream.cuh")
 
 
 def source_hash():
@@ -315,6 +390,217 @@ def job_gbs(world, bytes_per_step, steps, ms):
     return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
 
 
+def recorded_ncu_time(kernel_label, workload_name):
+    """ncu gpu__time_duration of one launch (cold L2, launches serialised)
+    from the committed profile record, while the kernel sources still match."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        e = json.load(f).get(workload_name, {}).get(kernel_label)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("ncu_us")
+
+
+def _graph(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def _time_graph(torch, g, min_ms):
+    """Average ms per replay of CUDA graph g: one warm replay, a one-replay
+    estimate, then enough replays for at least `min_ms` of device time."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    torch.cuda.synchronize()
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    one = max(a.elapsed_time(b), 1e-3)
+    reps = int(min(20000, max(3, -(-min_ms // one))))
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def measure_workload(name, args, torch, world, with_cpu):
+    """One workload on this GPU: the step time over exactly `--steps` steps,
+    each launch's time back to back and alone, the end-to-end step time and
+    the CPU oracle baseline.  Returns the JSON object of the workload."""
+    launches, cfg = workload(name)
+    step_bytes = sum(l.nbytes for l in launches)
+    # Inputs larger than L2: rotate weight copies so that more than twice the
+    # L2 capacity streams through between two reads of the same bytes.  Small
+    # workloads flush L2 before every step instead (outside the per-launch
+    # events, which then give the value).
+    flush = step_bytes < 64 * 2**20
+    copies = 1 if flush else max(2, -(-2 * L2_BYTES // step_bytes) + 1)
+    per = [copies if flush else max(copies, -(-2 * L2_BYTES // l.nbytes) + 1) for l in launches]
+    dw = DeviceWorkload(launches, per, torch)
+    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step(k):
+        if flush:
+            scrub.fill_(k & 0xFF)
+        dw.step(k)
+
+    for k in range(max(args.warmup, copies)):
+        step(k)
+    torch.cuda.synchronize()
+    # the timed steps replay CUDA graphs of the public API calls: graphs[c]
+    # is one step on weight copy c, cycle the `copies` steps of a rotation
+    graphs = [_graph(torch, lambda c=c: step(c)) for c in range(copies)]
+    cycle = _graph(torch, lambda: [step(c) for c in range(copies)])
+    for g in graphs:
+        g.replay()
+    cycle.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch)
+    torch.cuda.synchronize()
+    with sampler:
+        t0.record(stream)
+        for _ in range(K // copies):   # exactly K steps: whole rotations ...
+            cycle.replay()
+        for k in range(K % copies):    # ... then the remaining single steps
+            graphs[k].replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
+    del graphs, cycle
+
+    # Each launch alone, two ways, each replayed for at least --min-ms:
+    #  back to back: a graph of R launches of that kernel rotating its own
+    #    weight copies (more than twice L2 between reuses); a launch may be
+    #    scheduled while the previous one drains (programmatic dependent
+    #    launch), as in a decode loop;
+    #  isolated: a graph of R (L2 scrub, launch) pairs, minus a graph of the R
+    #    scrubs alone: every launch starts cold, behind a kernel that does not
+    #    let it start early.
+    chained, isolated = [], []
+    for i in range(len(launches)):
+        if flush:
+            chained.append(None)
+        else:
+            R = 3 * per[i]
+            g = _graph(torch, lambda i=i, R=R: [dw.run(i, r) for r in range(R)])
+            chained.append(max_over_ranks(_time_graph(torch, g, args.min_ms) / R, "cuda"))
+            del g
+        R = 8
+        g1 = _graph(torch, lambda i=i: [(scrub.fill_(r), dw.run(i, r)) for r in range(R)])
+        g2 = _graph(torch, lambda: [scrub.fill_(r) for r in range(R)])
+        d = (_time_graph(torch, g1, args.min_ms) - _time_graph(torch, g2, args.min_ms)) / R
+        isolated.append(max_over_ranks(d, "cuda"))
+        del g1, g2
+
+    # End to end through the public API: per step, the step's inputs in from
+    # pinned host memory (one copy), the launches, the outputs back to pinned
+    # host memory (one copy); one CUDA graph per step.
+    for k in range(copies):
+        dw.e2e_step(k)
+    torch.cuda.synchronize()
+    egraphs = [_graph(torch, lambda c=c: dw.e2e_step(c)) for c in range(copies)]
+    for g in egraphs:
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(K):
+        egraphs[k % copies].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
+    del egraphs
+
+    peak, peak_kind = measured_peaks()
+    out_launch = {}
+    basis = "isolated" if flush else "back to back"
+    us_of = []
+    for l, c, iso in zip(launches, chained, isolated):
+        d = iso if c is None else c
+        us_of.append(d)
+        gbs = l.nbytes / (d * 1e-3) / 1e9
+        out_launch[l.label] = {
+            "us": round(d * 1e3, 3), "us_back_to_back": None if c is None else round(c * 1e3, 3),
+            "us_isolated": round(iso * 1e3, 3), "us_basis": basis, "GB/s": round(gbs, 1),
+            "frac_of_measured_peak": round(gbs / peak, 4), "bytes": l.nbytes,
+            "ncu_us": recorded_ncu_time(l.label, name)}
+    dom = max(range(len(launches)), key=lambda i: us_of[i])
+    ach = launches[dom].nbytes / (us_of[dom] * 1e-3) / 1e9
+    value = job_gbs(world, step_bytes, K, ms)
+    if flush:   # the step region includes the L2 scrub: use kernel time only
+        value = world * step_bytes / (sum(isolated) * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 accumulate (bf16 in/out)" if name != "quantize" else "f32 (bf16 in/out)",
+        "data": "synthetic",
+        "config": dict(cfg, l2=(f"L2 flushed before every step ({2 * L2_BYTES >> 20} MiB "
+                                f"write); value from the isolated per-launch times" if flush else
+                                f"inputs larger than L2: {copies} rotating weight copies, "
+                                f"{step_bytes * copies / 2**20:.0f} MiB between reuse; each "
+                                f"launch timed back to back rotates through more than "
+                                f"{2 * L2_BYTES >> 20} MiB of its own copies"),
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       graphs=f"timed steps replayed as CUDA graphs of {copies} steps (one "
+                              f"weight rotation); the remainder one step per graph"),
+        "roofline": {"bound": "hbm", "kernel": launches[dom].label,
+                     "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "peak_kind": peak_kind,
+                     "timing": basis,
+                     "traffic": recorded_traffic(launches[dom].label, name),
+                     "algorithmic_bytes_per_launch": launches[dom].nbytes},
+        "per_launch": out_launch,
+        "tokens_per_s_equiv": {l.label: round(1e6 / (d * 1e3), 1)
+                               for l, d in zip(launches, us_of)},
+        "e2e": {"value": round(job_gbs(world, step_bytes, K, e2e_ms), 1),
+                "unit": UNIT, "h2d_bytes_per_step": dw.h2d_bytes,
+                "d2h_bytes_per_step": dw.d2h_bytes,
+                "note": "weights resident in HBM; each step's inputs copied in (one "
+                        "copy) and outputs copied out (one copy); each step replayed "
+                        "as one CUDA graph"},
+        "gpu_launches": K * len(launches),
+        "clocks": sampler.summary(),
+    }
+    if with_cpu:
+        budget = args.cpu_budget if name == args.workload else args.cpu_budget_config
+        res["cpu_baseline"] = cpu_baseline(launches, budget_s=budget)
+    del dw, scrub
+    torch.cuda.empty_cache()
+    return res
+
+
+def _spawn_replicas(args):
+    """`--gpus N` without torchrun: relaunch this command under torchrun, one
+    process per GPU, or stop with an error when fewer GPUs are visible."""
+    import subprocess
+    import torch
+    have = torch.cuda.device_count() if torch.cuda.is_available() else 0
+    if have < args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} needs {args.gpus} visible GPUs, "
+                         f"found {have}\n")
+        return 2
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={args.master_port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "moe_gather", "quantize")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -329,348 +615,14 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     import affine_group_quantized_b200 as agq
     agq.lib()
-
-    launches, cfg = workload(args.workload)
-    step_bytes = sum(l.nbytes for l in launches)
-    # Inputs larger than L2: rotate weight copies so that more than twice the
-    # L2 capacity streams through between two reads of the same bytes.  Small
-    # workloads instead flush L2 before every step (outside the per-launch
-    # events, which then give the value).
-    flush = step_bytes < 64 * 2**20
-    copies = 1 if flush else max(2, -(-2 * L2_BYTES // step_bytes) + 1)
-    # Each launch also gets enough weight copies that timing it alone (below)
-    # streams more than twice the L2 capacity between two reads of the same
-    # bytes; a step uses the first `copies` of them.
-    dls = [DeviceLaunch(l, copies if flush else max(copies, -(-2 * L2_BYTES // l.nbytes) + 1),
-                        torch) for l in launches]
-    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if flush else None
-
-    def step(k):
-        if scrub is not None:
-            scrub.fill_(k & 0xFF)
-        for dl in dls:
-            dl(k)
-
-    for k in range(max(args.warmup, copies)):
-        step(k)
-    torch.cuda.synchronize()
-
-    # Every timed region replays CUDA graphs captured from the public API
-    # calls, so the host's per-call enqueue cost does not pace the GPU.
-    # graphs[c] = one full step using weight copy c; cycle = the `copies`
-    # steps of one rotation in a single graph (fewer graph launches per
-    # step, as a decode loop captured whole would run).
-    graphs = []
-    for c in range(copies):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(c)
-        graphs.append(g)
-    cycle = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle):
-        for c in range(copies):
-            step(c)
-    for c in range(copies):
-        graphs[c].replay()
-    cycle.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-
-    K = args.steps
-    stream = torch.cuda.current_stream()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(torch)
-    torch.cuda.synchronize()
-    with sampler:
-        t0.record(stream)
-        for _ in range(K // copies):  # exactly K steps: whole rotations ...
-            cycle.replay()
-        for k in range(K % copies):   # ... then the remaining single steps
-            graphs[k].replay()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
-
-    # Average duration of each launch: a graph of R back-to-back launches of
-    # that kernel alone (rotating through all of its weight copies, more than
-    # twice the L2 capacity; L2 scrubbed first for the small workloads), timed
-    # with events around the replays.
-    dur = []
-    for dl in dls:
-        R = 3 * len(dl.copies)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for r in range(R):
-                if scrub is not None:
-                    scrub.fill_(r & 0xFF)
-                dl(r)
-        g.replay()
-        torch.cuda.synchronize()
-        reps = max(1, min(200, (K * len(dls)) // R))
-        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            g.replay()
-        b_.record(stream)
-        torch.cuda.synchronize()
-        d = a.elapsed_time(b_) / (reps * R)
-        if scrub is not None:  # remove the scrub's own time
-            gs_ = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gs_):
-                for r in range(R):
-                    scrub.fill_(r & 0xFF)
-            gs_.replay()
-            torch.cuda.synchronize()
-            a.record(stream)
-            for _ in range(reps):
-                gs_.replay()
-            b_.record(stream)
-            torch.cuda.synchronize()
-            d -= a.elapsed_time(b_) / (reps * R)
-        dur.append(d)
-
-    # End to end through the public API: per step, copy x in from pinned host
-    # memory, run the step's launches, copy y out to pinned host memory (one
-    # CUDA graph per step).
-    hx = [dl.x.detach().cpu().pin_memory() for dl in dls]
-    hy = [torch.empty_like(dl.y, device="cpu").pin_memory() for dl in dls]
-    h2d = sum(t.numel() * t.element_size() for t in hx)
-    d2h = sum(t.numel() * t.element_size() for t in hy)
-
-    def e2e_step(k):
-        for i, dl in enumerate(dls):
-            dl.x.copy_(hx[i], non_blocking=True)
-            dl(k)
-            hy[i].copy_(dl.y, non_blocking=True)
-
-    for k in range(copies):
-        e2e_step(k)
-    torch.cuda.synchronize()
-    egraphs = []
-    for c in range(copies):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            e2e_step(c)
-        egraphs.append(g)
-    for g in egraphs:
-        g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for k in range(K):
-        egraphs[k % copies].replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
-    del graphs, egraphs
-
-    peak, peak_kind = measured_peaks()
-    per = {}
-    for l, d in zip(launches, dur):
-        gbs = l.nbytes / (d * 1e-3) / 1e9
-        per[l.label] = {"us": round(d * 1e3, 3), "GB/s": round(gbs, 1),
-                        "frac_of_measured_peak": round(gbs / peak, 4),
-                        "bytes": l.nbytes}
-    dom = max(range(len(dls)), key=lambda i: dur[i])
-    ach = launches[dom].nbytes / (dur[dom] * 1e-3) / 1e9
-    value = job_gbs(world, step_bytes, K, ms)
-    if flush:  # the step region includes the L2 scrub: use kernel time only
-        value = world * step_bytes / (sum(dur) * 1e-3) / 1e9
-    out = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32 accumulate (bf16 in/out)", "data": "synthetic",
-        "config": dict(cfg, l2=(f"L2 flushed before every step ({2 * L2_BYTES >> 20} MiB "
-                                f"write); value from per-launch events" if flush else
-                                f"inputs larger than L2: {copies} rotating weight copies, "
-                                f"{step_bytes * copies / 2**20:.0f} MiB between reuse; each "
-                                f"launch timed alone rotates through more than "
-                                f"{2 * L2_BYTES >> 20} MiB of its own copies"),
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       graphs=f"timed steps replayed as CUDA graphs of {copies} steps (one "
-                              f"weight rotation); the remainder one step per graph"),
-        "roofline": {"bound": "hbm", "kernel": launches[dom].label,
-                     "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(ach / peak, 4), "peak_kind": peak_kind,
-                     "traffic": recorded_traffic(launches[dom].label, args.workload),
-                     "algorithmic_bytes_per_launch": launches[dom].nbytes},
-        "per_launch": per,
-        "tokens_per_s_equiv": {l.label: round(1e6 / (d * 1e3), 1)
-                               for l, d in zip(launches, dur)},
-        "e2e": {"value": round(job_gbs(world, step_bytes, K, e2e_ms), 1),
-                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "weights resident in HBM (decode); x copied in and y copied "
-                        "out every step; each step replayed as one CUDA graph"},
-        "gpu_launches": K * len(dls),
-        "clocks": sampler.summary(),
-        "source_hash": source_hash(),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(launches, budget_s=args.cpu_budget)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-
-
-def run_quant(args):
-    """GPU arm of the quantize workload: one step = affine_quantize of a bf16
-    matrix and affine_dequantize of a packed one.  Inputs rotate through
-    copies so that more than twice the L2 capacity streams between two reads
-    of the same bytes; the dequantize of step k reads the codes the quantize
-    of an earlier step wrote (copy k + 1), so it never reads L2-hot output."""
-    import torch
-    import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    import affine_group_quantized_b200 as agq
-    agq.lib()
-
-    launches, cfg = workload("quantize")
-    lq, ld = launches
-    N, K, bits, gs = lq.N, lq.K, lq.bits, lq.gs
-    step_bytes = lq.nbytes + ld.nbytes
-    copies = max(3, -(-2 * L2_BYTES // (2 * N * K)) + 1)
-    bf, i32, i16 = torch.bfloat16, torch.int32, torch.int16
-    W = [_dev(lq.w, torch) for _ in range(copies)]
-    Q = [_dev(ld.w, torch) for _ in range(copies)]
-    S = [_dev(ld.s, torch) for _ in range(copies)]
-    B = [_dev(ld.b, torch) for _ in range(copies)]
-    Y = torch.empty((N, K), dtype=bf, device="cuda")
-
-    def quant(k):
-        c = k % copies
-        agq.affine_quantize(W[c], Q[c], S[c], B[c], N, K, bits, gs)
-
-    def dequant(k):
-        c = (k + 1) % copies
-        agq.affine_dequantize(Q[c], S[c], B[c], Y, N, K, bits, gs)
-
-    def step(k):
-        quant(k)
-        dequant(k)
-
-    for k in range(max(args.warmup, copies)):
-        step(k)
-    torch.cuda.synchronize()
-    graphs = []
-    for c in range(copies):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(c)
-        graphs.append(g)
-    for g in graphs:
-        g.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-
-    Ks = args.steps
-    stream = torch.cuda.current_stream()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(torch)
-    torch.cuda.synchronize()
-    with sampler:
-        t0.record(stream)
-        for k in range(Ks):
-            graphs[k % copies].replay()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
-
-    # each kernel alone: a graph of 3 * copies back-to-back launches
-    dur = []
-    for fn in (quant, dequant):
-        R = 3 * copies
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for r in range(R):
-                fn(r)
-        g.replay()
-        torch.cuda.synchronize()
-        reps = max(1, min(100, 2 * Ks // R))
-        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            g.replay()
-        b_.record(stream)
-        torch.cuda.synchronize()
-        dur.append(a.elapsed_time(b_) / (reps * R))
-
-    # end to end: the bf16 matrix in from pinned host memory, quantize,
-    # dequantize the result, and the packed matrix and the bf16 round trip out
-    hw = W[0].detach().cpu().pin_memory()
-    outs = (Q[0], S[0], B[0], Y)
-    houts = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
-    h2d = hw.numel() * hw.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in houts)
-
-    def e2e_step():
-        W[0].copy_(hw, non_blocking=True)
-        agq.affine_quantize(W[0], Q[0], S[0], B[0], N, K, bits, gs)
-        agq.affine_dequantize(Q[0], S[0], B[0], Y, N, K, bits, gs)
-        for h, d in zip(houts, outs):
-            h.copy_(d, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    eg = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(eg):
-        e2e_step()
-    eg.replay()
-    torch.cuda.synchronize()
-    ek = max(3, min(Ks, 20))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(ek):
-        eg.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
-    del graphs, eg
-
-    peak, peak_kind = measured_peaks()
-    per = {}
-    for l, d in zip(launches, dur):
-        gbs = l.nbytes / (d * 1e-3) / 1e9
-        per[l.label] = {"us": round(d * 1e3, 3), "GB/s": round(gbs, 1),
-                        "frac_of_measured_peak": round(gbs / peak, 4), "bytes": l.nbytes}
-    dom = 0 if dur[0] >= dur[1] else 1
-    ach = launches[dom].nbytes / (dur[dom] * 1e-3) / 1e9
-    out = {
-        "metric": METRIC, "value": round(job_gbs(world, step_bytes, Ks, ms), 1),
-        "unit": UNIT, "n_gpus": world, "steps": Ks, "warmup": args.warmup,
-        "ms_per_step": round(ms / Ks, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 (bf16 in/out)", "data": "synthetic",
-        "config": dict(cfg, l2=f"inputs larger than L2: {copies} rotating copies of every "
-                               f"input; dequantize reads codes written one step earlier",
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       graphs="timed steps replayed as one CUDA graph per step"),
-        "roofline": {"bound": "hbm", "kernel": launches[dom].label, "achieved": round(ach, 1),
-                     "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
-                     "peak_kind": peak_kind,
-                     "traffic": recorded_traffic(launches[dom].label, "quantize"),
-                     "algorithmic_bytes_per_launch": launches[dom].nbytes},
-        "per_launch": per,
-        "e2e": {"value": round(job_gbs(world, step_bytes, ek, e2e_ms), 1), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "bf16 matrix copied in, packed matrix and round trip copied out "
-                        "every step; each step replayed as one CUDA graph"},
-        "gpu_launches": 2 * Ks,
-        "clocks": sampler.summary(),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(launches, budget_s=args.cpu_budget)
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    out = measure_workload(args.workload, args, torch, world, with_cpu)
+    if args.configs == "all":
+        out["per_config"] = {}
+        for name in ALL_WORKLOADS:
+            if name != args.workload:
+                out["per_config"][name] = measure_workload(name, args, torch, world, with_cpu)
+    out["source_hash"] = source_hash()
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -693,9 +645,7 @@ def _oracle_launch(l, rows, nthreads):
         oracle.qmv(l.x, l.wu, l.su, l.bu, l.M, l.N, l.K, l.bits, l.gs, rows=rows,
                    nthreads=nthreads)
     elif l.kind == "silu":
-        g = synth.normal_bf16((l.M, l.K), seed=3004)
-        u = synth.normal_bf16((l.M, l.K), seed=3005)
-        oracle.silu_gate_resid(g, u, l.resid, l.w, l.s, l.b, l.M, l.N, l.K, l.bits,
+        oracle.silu_gate_resid(l.gate, l.up, l.resid, l.w, l.s, l.b, l.M, l.N, l.K, l.bits,
                                l.gs, rows=rows, nthreads=nthreads)
     elif l.kind == "gather":
         oracle.gather(l.x, l.w, l.s, l.b, l.lhs, l.rhs, l.P, l.T, l.E, l.N, l.K,
@@ -797,27 +747,36 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_sweep",
-                    choices=["decode_sweep", "qmv_small", "ffn_int8", "batched",
-                             "moe_gather", "quantize"])
+    ap.add_argument("--workload", default="decode_sweep", choices=list(ALL_WORKLOADS))
+    ap.add_argument("--configs", default="all", choices=["all", "none"],
+                    help="also measure every other workload (per_config)")
+    ap.add_argument("--min-ms", type=float, default=100.0,
+                    help="device time each per-launch timing graph is replayed for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    args = ap.parse_args()
+    ap.add_argument("--cpu-budget-config", type=float, default=6.0)
+    ap.add_argument("--master-port", type=int, default=29533)
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    world = os.environ.get("WORLD_SIZE")
+    if world is not None and int(world) != args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}\n")
+        return 2
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "quantize":
-        run_quant(args)
-    else:
-        run_ours(args)
+        return 0
+    if args.gpus > 1 and world is None:
+        return _spawn_replicas(args)
+    run_ours(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

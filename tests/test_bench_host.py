@@ -181,3 +181,34 @@ def test_committed_traffic_names_known_launches():
         assert set(entries) <= labels, name
         for e in entries.values():
             assert e["dram_bytes_per_launch"] > 0 and len(e["source_hash"]) == 16
+
+
+def test_gpus_flag_without_torchrun_needs_that_many_gpus(monkeypatch, capsys):
+    # `--gpus 2` outside torchrun relaunches under torchrun only when two GPUs
+    # are visible; on a box with fewer it stops with an error, never printing
+    # a one-GPU line
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    import torch
+    if torch.cuda.is_available() and torch.cuda.device_count() >= 2:
+        pytest.skip("two GPUs visible: the flag would launch the replicas")
+    assert bench.main(["--gpus", "2", "--steps", "3"]) == 2
+    err = capsys.readouterr().err
+    assert "--gpus 2 needs 2 visible GPUs" in err
+
+
+def test_gpus_flag_must_match_the_launcher(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    assert bench.main(["--gpus", "2"]) == 2
+    assert "WORLD_SIZE=4" in capsys.readouterr().err
+
+
+@pytest.mark.parametrize("name", bench.ALL_WORKLOADS)
+def test_every_workload_has_inputs_outputs_and_weights(name):
+    # the packed per-step input and output buffers cover every array the
+    # launches read per step and write
+    launches, _ = bench.workload(name)
+    for l in launches:
+        for k in bench._WEIGHTS[l.kind] + bench._INPUTS[l.kind]:
+            assert getattr(l, k) is not None, (l.label, k)
+        outs = bench._outputs(l)
+        assert outs and all(int(np.prod(s)) > 0 for _, s, _ in outs)
