@@ -9,11 +9,12 @@
 // CUDA cores with 16-byte coalesced loads and stores and a grid-stride loop
 // over one wave of resident blocks on every SM.
 //
-// Work unit: a "chunk" of 8 consecutive codes of the flattened [N, K]
-// matrix.  8 codes of `bits` bits are exactly `bits` bytes of the packed
-// stream (byte offset chunk * bits), and 8 bf16 weights are one 16-byte
-// vector, so a chunk is the natural unit for both directions.  Groups
-// (group_size in {32, 64, 128}) are whole numbers of chunks.
+// Work units: the quantizer gives each lane a "chunk" of 8 consecutive codes
+// of the flattened [N, K] matrix: 8 bf16 weights are one 16-byte load and 8
+// codes of `bits` bits are exactly `bits` bytes of the packed stream (byte
+// offset chunk * bits).  The dequantizer gives each thread "units" of 32
+// codes: `bits` whole packed words in, 64 bytes of bf16 out.  Groups
+// (group_size in {32, 64, 128}) are whole numbers of chunks and of units.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -36,22 +37,80 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) {
 // Dequantize: out = bf16(scale * q + bias), the exact value rounded once
 // ---------------------------------------------------------------------------
 
-// scale * q is exact in binary32 (8 by 8 significant bits), so one fused
-// multiply-add rounds the exact scale * q + bias once to binary32 (r).  r
-// rounds to bf16 exactly as the exact sum would, except when r lies exactly
-// halfway between two bf16 values (its low 16 bits are 0x8000) while the sum
-// was not exact: there the exact sum lies on the side of the two-sum error e,
-// which the rare slow path recovers.
-__device__ __noinline__ uint16_t affine_tie_to_bf16(float q, float s, float b, float r) {
-  const float p = __fmul_rn(q, s);
-  const float bv = __fsub_rn(r, p);
-  const float av = __fsub_rn(r, bv);
-  const float e = __fadd_rn(__fsub_rn(p, av), __fsub_rn(b, bv));
-  const uint32_t u = __float_as_uint(r);
-  if (e == 0.0f) return __bfloat16_as_ushort(__float2bfloat16_rn(r));  // a true tie
-  // sign-magnitude: adding 1 to the upper half grows the magnitude
-  const bool away = (e > 0.0f) == (r > 0.0f);
-  return static_cast<uint16_t>((u >> 16) + (away ? 1u : 0u));
+// The bf16 fused multiply-add computes s * q + b exactly and rounds once to
+// bf16 (nearest, ties to even), which is the definition itself.  The code q
+// enters as an exact bf16 value: for q < 128, the bits 0x4300 | q are the
+// bf16 number 128 + q, and subtracting 128 is exact; 8-bit codes (up to 255)
+// go through binary32 (0x4b000000 | q is 2^23 + q) and an exact conversion.
+__device__ __forceinline__ __nv_bfloat162 bf162_bits(uint32_t v) {
+  __nv_bfloat162 h;
+  *reinterpret_cast<uint32_t *>(&h) = v;
+  return h;
+}
+__device__ __forceinline__ uint32_t bf162_u32(__nv_bfloat162 h) {
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Dequantize works in units of 32 codes: exactly BITS packed words (4 * BITS
+// bytes at a multiple of 4 * BITS, loaded with the widest aligned loads),
+// always inside one group, and 64 bytes of bf16 output (four 16-byte
+// stores).  Each thread takes two units per pass, both loaded before either
+// is computed, so every thread keeps two loads in flight.
+template <int BITS>
+__device__ __forceinline__ void load_unit_words(const uint32_t *__restrict__ wq, long long u,
+                                                uint32_t (&w)[BITS]) {
+  const uint32_t *p = wq + u * BITS;
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS / 4; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS / 2; ++i) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p) + i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) w[i] = __ldg(p + i);
+  }
+}
+
+// Code i of a unit: bits [i * BITS, (i + 1) * BITS) of its little-endian
+// stream, taken with a funnel shift where it straddles two words.
+template <int BITS>
+__device__ __forceinline__ uint32_t unit_code(const uint32_t (&w)[BITS], int i) {
+  const int o = i * BITS, j = o >> 5, sh = o & 31;
+  const uint32_t v = (sh + BITS > 32) ? __funnelshift_r(w[j], w[j + 1], sh) : (w[j] >> sh);
+  return v & ((1u << BITS) - 1u);
+}
+
+// Codes 2j and 2j + 1 of a unit as an exact bf16 pair (code 2j low).
+template <int BITS>
+__device__ __forceinline__ __nv_bfloat162 code_pair(const uint32_t (&w)[BITS], int j) {
+  const uint32_t c0 = unit_code<BITS>(w, 2 * j), c1 = unit_code<BITS>(w, 2 * j + 1);
+  if constexpr (BITS == 8) {
+    const float f0 = __fsub_rn(__uint_as_float(0x4b000000u | c0), 8388608.0f);
+    const float f1 = __fsub_rn(__uint_as_float(0x4b000000u | c1), 8388608.0f);
+    return __floats2bfloat162_rn(f0, f1);  // exact: integers below 256
+  } else {
+    return __hsub2(bf162_bits(c0 | (c1 << 16) | 0x43004300u), bf162_bits(0x43004300u));
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void dequantize_unit(const uint32_t (&w)[BITS], uint32_t sb,
+                                                uint32_t bb, uint4 *__restrict__ dst) {
+  const __nv_bfloat162 s2 = bf162_bits(sb | (sb << 16)), b2 = bf162_bits(bb | (bb << 16));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {  // 8 codes per 16-byte store
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = bf162_u32(__hfma2(code_pair<BITS>(w, 4 * c + j), s2, b2));
+    dst[c] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
 }
 
 template <int BITS>
@@ -59,50 +118,26 @@ __global__ void __launch_bounds__(kThreads)
 affine_dequantize_kernel(const uint32_t *__restrict__ wq,
                          const uint16_t *__restrict__ scales,
                          const uint16_t *__restrict__ biases,
-                         uint4 *__restrict__ out, long long nchunks,
+                         uint4 *__restrict__ out, long long nunits,
                          int gs_shift) {
-  constexpr uint32_t kMask = (1u << BITS) - 1u;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-       c < nchunks; c += stride) {
-    // the chunk's `BITS` bytes start at byte c * BITS; with at most 3 bytes
-    // of offset into the first word they end within the next word
-    const long long byte0 = c * BITS;
-    const long long w0 = byte0 >> 2;
-    const int off = static_cast<int>(byte0 & 3);
-    uint64_t v = __ldg(wq + w0);
-    if (off + BITS > 4) v |= static_cast<uint64_t>(__ldg(wq + w0 + 1)) << 32;
-    v >>= 8 * off;
-    const long long g = (c * 8) >> gs_shift;
-    const float s = bf16_bits_to_float(__ldg(scales + g));
-    const float b = bf16_bits_to_float(__ldg(biases + g));
-    float q[8], r[8];
-    bool tie = false;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      // the code as an exact float: 2^23 + q has q in its low mantissa bits
-      const uint32_t code = static_cast<uint32_t>(v >> (BITS * i)) & kMask;
-      q[i] = __fsub_rn(__uint_as_float(0x4b000000u | code), 8388608.0f);
-      r[i] = __fmaf_rn(q[i], s, b);
-      tie |= (__float_as_uint(r[i]) & 0xffffu) == 0x8000u;
+  for (long long u0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+       u0 < nunits; u0 += 2 * stride) {
+    const long long u1 = u0 + stride;
+    const bool two = u1 < nunits;
+    uint32_t w0[BITS], w1[BITS];
+    load_unit_words<BITS>(wq, u0, w0);
+    const long long g0 = (u0 * 32) >> gs_shift;
+    const uint32_t s0 = __ldg(scales + g0), b0 = __ldg(biases + g0);
+    uint32_t s1 = 0, b1 = 0;
+    if (two) {
+      load_unit_words<BITS>(wq, u1, w1);
+      const long long g1 = (u1 * 32) >> gs_shift;
+      s1 = __ldg(scales + g1);
+      b1 = __ldg(biases + g1);
     }
-    uint32_t h[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat162 pr = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
-      h[j] = *reinterpret_cast<const uint32_t *>(&pr);
-    }
-    if (tie) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if ((__float_as_uint(r[i]) & 0xffffu) == 0x8000u) {
-          const uint32_t hi = affine_tie_to_bf16(q[i], s, b, r[i]);
-          const int sh = 16 * (i & 1);
-          h[i >> 1] = (h[i >> 1] & ~(0xffffu << sh)) | (hi << sh);
-        }
-      }
-    }
-    out[c] = make_uint4(h[0], h[1], h[2], h[3]);
+    dequantize_unit<BITS>(w0, s0, b0, out + 4 * u0);
+    if (two) dequantize_unit<BITS>(w1, s1, b1, out + 4 * u1);
   }
 }
 
@@ -136,63 +171,100 @@ __device__ __forceinline__ void store_chunk(uint8_t *wq, long long c, uint64_t p
 // iteration (the loop bound is uniform over the warp); lanes past the end
 // load nothing and store nothing, and since the chunk count is a whole number
 // of groups they never share a group with a live lane.
+// The code of one element: min(round(d / scale), n_bins) with the page's
+// binary32 quotient d / scale and round-half-away.  The quotient is formed
+// as d * (1 / scale) (both correctly rounded), within 3 * 2^-24 of the
+// binary32 quotient relative to it; where no half-integer lies within
+// 2^-20 * max(|t|, 1) of that product, both round to the same integer and
+// rint gives it.  Only the rare elements near a half-integer take the IEEE
+// division and roundf, so every code is the one the page's steps decide.
+__device__ __forceinline__ uint32_t quantize_code(float v, float bias, float scale, float rcp,
+                                                  float n_bins) {
+  const float d = __fsub_rn(v, bias);
+  const float tp = __fmul_rn(d, rcp);
+  const float rt = rintf(tp);
+  float code = rt;
+  if (fabsf(__fsub_rn(tp, rt)) > 0.5f - fmaxf(fabsf(tp), 1.0f) * 0x1p-20f)
+    code = roundf(__fdiv_rn(d, scale));
+  return static_cast<uint32_t>(fminf(code, n_bins));
+}
+
+// One work item: 32 chunks (one warp, lane = chunk).  Computes the group
+// parameters with xor butterflies over the group's lanes, stores the group's
+// scale and bias from its first lane and the lane's packed codes.
+template <int BITS, int GS>
+__device__ __forceinline__ void quantize_item(const uint4 raw, long long c, bool live, int lane,
+                                              uint8_t *__restrict__ wq,
+                                              uint16_t *__restrict__ scales,
+                                              uint16_t *__restrict__ biases) {
+  constexpr int kLanes = GS / 8;  // lanes per group
+  const float n_bins = static_cast<float>((1 << BITS) - 1);
+  const float eps = 1e-7f;
+  const float start_min = bf16_bits_to_float(0x7f7fu);  // largest finite bf16
+  const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(pr[i] << 16);
+    v[2 * i + 1] = __uint_as_float(pr[i] & 0xffff0000u);
+  }
+  float w_min = start_min, w_max = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    w_min = fminf(w_min, v[i]);
+    w_max = fmaxf(w_max, v[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < kLanes; o <<= 1) {
+    w_min = fminf(w_min, __shfl_xor_sync(0xffffffffu, w_min, o));
+    w_max = fmaxf(w_max, __shfl_xor_sync(0xffffffffu, w_max, o));
+  }
+  float scale = fmaxf(__fdiv_rn(__fsub_rn(w_max, w_min), n_bins), eps);
+  const bool side = fabsf(w_min) > fabsf(w_max);
+  scale = side ? scale : -scale;
+  const float edge = side ? w_min : w_max;
+  const float q0 = roundf(__fdiv_rn(edge, scale));
+  const bool at_zero = q0 == 0.0f;
+  scale = at_zero ? scale : __fdiv_rn(edge, q0);
+  const float bias = at_zero ? 0.0f : edge;
+  if (live && (lane % kLanes) == 0) {
+    const long long g = c / kLanes;
+    scales[g] = __bfloat16_as_ushort(__float2bfloat16_rn(scale));
+    biases[g] = __bfloat16_as_ushort(__float2bfloat16_rn(bias));
+  }
+  const float rcp = __frcp_rn(scale);
+  uint64_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    packed |= static_cast<uint64_t>(quantize_code(v[i], bias, scale, rcp, n_bins)) << (BITS * i);
+  if (live) store_chunk<BITS>(wq, c, packed);
+}
+
+// One lane per chunk; the GS / 8 lanes of a group are consecutive, and a
+// work item's 32 chunks start on a group boundary, so the group's min and
+// max are butterfly reductions inside those lanes.  All 32 lanes run every
+// item (the loop bound is uniform over the warp); lanes past the end load
+// nothing and store nothing, and since the chunk count is a whole number of
+// groups they never share a group with a live lane.  A warp takes two items
+// per pass (items wi and wi + warps), both loaded before either is computed.
 template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads)
 affine_quantize_kernel(const uint4 *__restrict__ w, uint8_t *__restrict__ wq,
                        uint16_t *__restrict__ scales,
                        uint16_t *__restrict__ biases, long long nchunks) {
-  constexpr int kLanes = GS / 8;  // lanes per group
-  const float n_bins = static_cast<float>((1 << BITS) - 1);
-  const float eps = 1e-7f;
-  const float start_min = bf16_bits_to_float(0x7f7fu);  // largest finite bf16
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
   const long long nwork = (nchunks + 31) / 32;
   for (long long wi = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-       wi < nwork; wi += warps) {
-    const long long c = wi * 32 + lane;
-    const bool live = c < nchunks;
-    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-    if (live) raw = __ldg(w + c);
-    const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(pr[i] << 16);
-      v[2 * i + 1] = __uint_as_float(pr[i] & 0xffff0000u);
-    }
-    float w_min = start_min, w_max = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      w_min = fminf(w_min, v[i]);
-      w_max = fmaxf(w_max, v[i]);
-    }
-#pragma unroll
-    for (int o = 1; o < kLanes; o <<= 1) {
-      w_min = fminf(w_min, __shfl_xor_sync(0xffffffffu, w_min, o));
-      w_max = fmaxf(w_max, __shfl_xor_sync(0xffffffffu, w_max, o));
-    }
-    float scale = fmaxf(__fdiv_rn(__fsub_rn(w_max, w_min), n_bins), eps);
-    const bool side = fabsf(w_min) > fabsf(w_max);
-    scale = side ? scale : -scale;
-    const float edge = side ? w_min : w_max;
-    const float q0 = roundf(__fdiv_rn(edge, scale));
-    const bool at_zero = q0 == 0.0f;
-    scale = at_zero ? scale : __fdiv_rn(edge, q0);
-    const float bias = at_zero ? 0.0f : edge;
-    if (live && (lane % kLanes) == 0) {
-      const long long g = c / kLanes;
-      scales[g] = __bfloat16_as_ushort(__float2bfloat16_rn(scale));
-      biases[g] = __bfloat16_as_ushort(__float2bfloat16_rn(bias));
-    }
-    uint64_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float t = __fdiv_rn(__fsub_rn(v[i], bias), scale);
-      const uint32_t q = static_cast<uint32_t>(fminf(roundf(t), n_bins));
-      packed |= static_cast<uint64_t>(q) << (BITS * i);
-    }
-    if (live) store_chunk<BITS>(wq, c, packed);
+       wi < nwork; wi += 2 * warps) {
+    const long long c0 = wi * 32 + lane, c1 = (wi + warps) * 32 + lane;
+    const bool live0 = c0 < nchunks, live1 = c1 < nchunks;
+    const bool item1 = wi + warps < nwork;  // warp-uniform
+    uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
+    if (live0) r0 = __ldg(w + c0);
+    if (live1) r1 = __ldg(w + c1);
+    quantize_item<BITS, GS>(r0, c0, live0, lane, wq, scales, biases);
+    if (item1) quantize_item<BITS, GS>(r1, c1, live1, lane, wq, scales, biases);
   }
 }
 
@@ -264,8 +336,9 @@ int launch_quantize_gs(cudaStream_t st, const uint4 *w, uint8_t *wq, uint16_t *s
                        uint16_t *b, long long nchunks) {
   constexpr auto kern = qmvq::affine_quantize_kernel<BITS, GS>;
   int grid = 0;
-  // one warp per 32 chunks, kThreads / 32 warps per block
-  int rc = launch_grid((nchunks + 31) / 32, qmvq::kThreads / 32, resident_blocks<kern>(), &grid);
+  // one warp per two items of 32 chunks, kThreads / 32 warps per block
+  int rc = launch_grid(((nchunks + 31) / 32 + 1) / 2, qmvq::kThreads / 32,
+                       resident_blocks<kern>(), &grid);
   if (rc) return rc;
   kern<<<grid, qmvq::kThreads, 0, st>>>(w, wq, s, b, nchunks);
   cudaError_t e = cudaGetLastError();
@@ -287,9 +360,11 @@ int launch_dequantize(int gs_shift, cudaStream_t st, const uint32_t *wq, const u
                       const uint16_t *b, uint4 *out, long long nchunks) {
   constexpr auto kern = qmvq::affine_dequantize_kernel<BITS>;
   int grid = 0;
-  int rc = launch_grid(nchunks, qmvq::kThreads, resident_blocks<kern>(), &grid);
+  // two 32-code units per thread and pass
+  const long long nunits = nchunks / 4;
+  int rc = launch_grid((nunits + 1) / 2, qmvq::kThreads, resident_blocks<kern>(), &grid);
   if (rc) return rc;
-  kern<<<grid, qmvq::kThreads, 0, st>>>(wq, s, b, out, nchunks, gs_shift);
+  kern<<<grid, qmvq::kThreads, 0, st>>>(wq, s, b, out, nunits, gs_shift);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return qfail(QMV_ERR_CUDA, "affine_dequantize launch: %s", cudaGetErrorString(e));

@@ -1,78 +1,64 @@
-"""CPU model of the dequantize kernel's rounding, checked against exact
-rational arithmetic.
+"""CPU checks of the dequantize kernel's arithmetic.
 
-The kernel forms r = scale * q + bias with one fused multiply-add (the
-product is exact in binary32, so r is the exact sum rounded once to
-binary32) and converts r to bf16 with round-to-nearest-even, except when r
-lies exactly halfway between two bf16 values: then the two-sum error of the
-addition says on which side the exact sum lies.  This test applies exactly
-those steps with numpy and Python fractions (no GPU, no kernel code) and
-asserts that the result is the exact sum rounded once to bf16, on random
-inputs and on constructed ties; without the tie step some of those cases
-round the wrong way, so the check is not vacuous.
+The kernel forms each output with one bf16 fused multiply-add,
+bf16(scale * q + bias) with a single rounding (nearest, ties to even), which
+is the definition of the dequantized weight itself.  Its only other step is
+turning a code q into an exact bf16 operand:
+  * codes below 128 (2- to 6-bit): the bits 0x4300 | q are the bf16 number
+    128 + q, and subtracting 128 is exact;
+  * 8-bit codes: the binary32 bits 0x4b000000 | q are 2^23 + q, subtracting
+    2^23 is exact, and the integer (below 256) converts to bf16 exactly.
+These tests check both encodings for every code with plain bit arithmetic
+and exact rationals, and that the exact value rounded once to bf16 is what
+the oracle's dequantizer returns (so a kernel computing it matches the
+oracle bit for bit).
 """
 from fractions import Fraction
 
 import numpy as np
 
+import oracle
 from tests._codes import exact_bf16 as _exact_bf16
 
 
-def _f32(x: Fraction) -> Fraction:
-    # binary32 rounding of an exact value (via binary64, exact for these
-    # inputs: a bf16 times a code below 256 plus a bf16 within 2^40 of it)
-    d = float(x)
-    assert Fraction(d) == x
-    return Fraction(float(np.float32(d)))
+def _bf16_value(bits: int) -> Fraction:
+    return Fraction(float(np.array([bits << 16], dtype=np.uint32).view(np.float32)[0]))
 
 
-def _bf16_rne_of_f32(r: Fraction) -> int:
-    u = int(np.array([float(r)], dtype=np.float32).view(np.uint32)[0])
-    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) & 0xFFFF
+def test_small_codes_encode_exactly_in_bf16():
+    for q in range(128):
+        assert _bf16_value(0x4300 | q) == 128 + q
+        # the difference with 128 is exactly q, so the subtraction is exact
+        assert _exact_bf16(_bf16_value(0x4300 | q) - 128) == _exact_bf16(Fraction(q))
+    assert _bf16_value(0x4300) == 128
 
 
-def _model(s: Fraction, q: int, b: Fraction, tie_step=True) -> int:
-    exact = s * q + b
-    r = _f32(exact)
-    u = int(np.array([float(r)], dtype=np.float32).view(np.uint32)[0])
-    if tie_step and (u & 0xFFFF) == 0x8000 and exact != r:
-        away = (exact > r) == (r > 0)
-        return ((u >> 16) + (1 if away else 0)) & 0xFFFF
-    return _bf16_rne_of_f32(r)
+def test_eight_bit_codes_encode_exactly_via_binary32():
+    for q in range(256):
+        f = np.array([0x4B000000 | q], dtype=np.uint32).view(np.float32)[0]
+        v = np.float32(f - np.float32(8388608.0))
+        assert Fraction(float(v)) == q
+        # an integer below 256 has at most 8 significant bits: exact in bf16
+        assert _bf16_value(_exact_bf16(Fraction(q))) == q
 
 
-def _bf16(v) -> Fraction:
-    return Fraction(float(v))
-
-
-def test_model_rounds_like_the_exact_sum_on_random_inputs():
+def test_single_rounding_is_the_oracles_dequantized_value():
+    # the oracle's dequantizer rounds the exact scale * q + bias once to bf16;
+    # so does one bf16 fused multiply-add, whatever the inputs
     rng = np.random.default_rng(17)
-    for _ in range(4000):
-        s = _bf16(np.ldexp(float(rng.integers(128, 256)) * rng.choice([-1, 1]),
-                           int(rng.integers(-30, 10))))
-        b = _bf16(np.ldexp(float(rng.integers(128, 256)) * rng.choice([-1, 1]),
-                           int(rng.integers(-30, 10))))
-        q = int(rng.integers(0, 256))
-        assert _model(s, q, b) == _exact_bf16(s * q + b)
-
-
-def test_model_on_binary32_ties():
-    # s * q exactly halfway between two bf16 values, with a bias small
-    # enough that binary32 rounds the sum back onto the halfway point
-    cases = 0
-    wrong_without = 0
-    for m in range(129, 256, 2):                 # odd 8-bit significands
-        s = Fraction(m, 128)
-        for q in (3, 5, 7, 9, 129, 255):
-            p = s * q
-            for eb in (-40, -35, -30):
-                for sign in (1, -1, 0):
-                    b = Fraction(sign) * Fraction(2) ** eb
-                    exact = p + b
-                    if _f32(exact) != _f32(p):
-                        continue
-                    cases += 1
-                    want = _exact_bf16(exact)
-                    assert _model(s, q, b) == want
-                    wrong_without += _model(s, q, b, tie_step=False) != want
-    assert cases > 100 and wrong_without > 0
+    N, K, bits, gs = 4, 64, 4, 32
+    G = K // gs
+    codes = rng.integers(0, 1 << bits, size=(N, K))
+    sb = rng.integers(0, 1 << 16, size=(N, G)).astype(np.uint16)
+    bb = rng.integers(0, 1 << 16, size=(N, G)).astype(np.uint16)
+    # keep finite, moderate magnitudes (exponent field 100..150)
+    sb = (sb & 0x807F) | (rng.integers(100, 150, size=(N, G)).astype(np.uint16) << 7)
+    bb = (bb & 0x807F) | (rng.integers(100, 150, size=(N, G)).astype(np.uint16) << 7)
+    from tests._codes import pack
+    w = pack(codes, bits)
+    got = oracle.dequantize_bf16(w, sb, bb, N, K, bits, gs)
+    for n in range(N):
+        for k in range(K):
+            g = k // gs
+            exact = _bf16_value(int(sb[n, g])) * int(codes[n, k]) + _bf16_value(int(bb[n, g]))
+            assert int(got[n, k]) == _exact_bf16(exact), (n, k)

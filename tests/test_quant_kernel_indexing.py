@@ -26,37 +26,59 @@ def _gs_ok(K, gs):
 
 @pytest.mark.parametrize("bits", ALL_BITS)
 @pytest.mark.parametrize("gs", [32, 64, 128])
-def test_dequantize_chunks_read_their_codes(bits, gs):
+def test_dequantize_units_read_their_codes(bits, gs):
+    # a dequantize unit is 32 codes: words [u*bits, (u+1)*bits) of the packed
+    # stream; code i of the unit is bits [i*bits, (i+1)*bits) of those words
+    # (a funnel shift of words j, j+1 where it straddles them); its group is
+    # (32u) >> gs_shift and its output is the 64 bytes of elements [32u, 32u+32)
     gs_shift = {32: 5, 64: 6, 128: 7}[gs]
     rng = np.random.default_rng(bits * 131 + gs)
+    mask = (1 << bits) - 1
     for N, K in SHAPES:
         if not _gs_ok(K, gs):
             continue
         codes = rng.integers(0, 1 << bits, size=(N, K))
         words = pack(codes, bits).reshape(-1).astype(np.uint64)
-        nwords = words.size
-        nchunks = N * K // 8
-        c = np.arange(nchunks, dtype=np.int64)
-        byte0 = c * bits
-        w0 = byte0 >> 2
-        off = byte0 & 3
-        need2 = off + bits > 4
-        assert w0.max() < nwords
-        assert (w0[need2] + 1).max(initial=0) < nwords
-        # the chunk's bytes lie inside the words it loads
-        last_byte = byte0 + bits - 1
-        assert np.all((last_byte >> 2) == np.where(need2, w0 + 1, w0))
-        v = words[w0].copy()
-        v[need2] |= words[w0[need2] + 1] << np.uint64(32)
-        v >>= (8 * off).astype(np.uint64)
-        mask = np.uint64((1 << bits) - 1)
-        got = np.stack([(v >> np.uint64(bits * i)) & mask for i in range(8)], axis=1)
+        nunits = N * K // 32
+        assert nunits * 32 == N * K
+        u = np.arange(nunits, dtype=np.int64)
+        first = u * bits
+        assert (first + bits - 1).max() < words.size        # loads stay inside
+        # the widest aligned loads: 16 bytes for 4/8-bit, 8 for 2/6, 4 for 3/5
+        align = 16 if bits % 4 == 0 else 8 if bits % 2 == 0 else 4
+        assert np.all((first * 4) % align == 0)
+        got = np.zeros((nunits, 32), dtype=np.int64)
+        for i in range(32):
+            o = i * bits
+            j, sh = o >> 5, o & 31
+            lo = words[first + j] >> np.uint64(sh)
+            if sh + bits > 32:
+                assert j + 1 < bits                          # the next word is the unit's
+                lo |= words[first + j + 1] << np.uint64(32 - sh)
+            got[:, i] = (lo & np.uint64(mask)).astype(np.int64)
         assert np.array_equal(got.reshape(N, K), codes)
-        g = (c * 8) >> gs_shift
+        g = (u * 32) >> gs_shift
         assert g.max() < N * (K // gs)
-        assert np.array_equal(g, (c * 8) // gs)
-        # the 16-byte output vector of chunk c covers elements [8c, 8c + 8)
-        assert (c.max() + 1) * 8 == N * K
+        assert np.array_equal(g, (u * 32) // gs)
+        # a unit never spans two groups
+        assert np.array_equal(((u * 32 + 31) >> gs_shift), g)
+
+
+@pytest.mark.parametrize("units, grid, per_block", [
+    (1, 1, 256), (301, 2, 256), (4097, 3, 8), (100001, 888, 8), (7, 888, 256)])
+def test_dequantize_two_units_per_pass_visit_each_unit_once(units, grid, per_block):
+    # thread t takes units u0 = t + 2*stride*k and u0 + stride (when below
+    # the count) on pass k
+    stride = grid * per_block
+    seen = np.zeros(units, dtype=np.int64)
+    for t in range(stride):
+        u0 = t
+        while u0 < units:
+            seen[u0] += 1
+            if u0 + stride < units:
+                seen[u0 + stride] += 1
+            u0 += 2 * stride
+    assert (seen == 1).all()
 
 
 def _grid_stride_visits(n_items, grid, per_block):
@@ -89,6 +111,16 @@ def test_quantize_lanes_groups_and_stores(bits, gs):
         written = np.zeros(nbytes, dtype=np.int64)
         sgroups = np.zeros(ngroups, dtype=np.int64)
         nwork = (nchunks + 31) // 32
+        # a warp takes items wi and wi + warps per pass; every item is visited
+        # once whatever the warp count
+        for warps in (1, 3, 8):
+            seen = np.zeros(nwork, dtype=np.int64)
+            for w0 in range(warps):
+                for wi in range(w0, nwork, 2 * warps):
+                    seen[wi] += 1
+                    if wi + warps < nwork:
+                        seen[wi + warps] += 1
+            assert (seen == 1).all()
         for wi in range(nwork):
             c = wi * 32 + np.arange(32)
             live = c < nchunks
