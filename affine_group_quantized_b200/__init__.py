@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.qmv_last_error.argtypes = []
         L.qmv_abi_version.restype = I
         L.qmv_abi_version.argtypes = []
+        L.qvm.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+        L.qvm.restype = I
         L.qmv_device_status.argtypes = [P, I, P]
         L.qmv_device_status.restype = I
         L.affine_quantize.argtypes = [P, P, P, P, I, I, I, I, P]
@@ -76,7 +78,7 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-EXPORTED = ("qmv", "qmv_noalloc", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
+EXPORTED = ("qmv", "qmv_noalloc", "qvm", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
             "qmv_last_error", "qmv_abi_version", "qmv_device_status", "affine_quantize",
             "affine_dequantize", "qmv_quant_last_error")
 
@@ -87,6 +89,26 @@ def _ptr(a):
     if isinstance(a, int):
         return a
     return a.data_ptr()
+
+
+def _need(name, t, nbytes):
+    """A tensor argument must hold at least the bytes the call reads or
+    writes (plain integer addresses are the caller's responsibility)."""
+    if t is None or isinstance(t, int):
+        return
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name}: {have} bytes, the call needs {nbytes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _need_qmv(rows, codes, bits, gs, **arrays):
+    """Sizes of a packed weight set: w [rows, codes*bits/32] uint32, scales
+    and biases [rows, codes/gs] bf16."""
+    _need("w", arrays.get("w"), rows * codes * bits // 8)
+    for k in ("scales", "biases"):
+        _need(k, arrays.get(k), 2 * rows * (codes // max(gs, 1)))
 
 
 def _stream(stream):
@@ -127,20 +149,35 @@ def device_status(reset=False, stream=None) -> int:
 
 def qmv(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):
     """y[M,N] = x[M,K] @ dequant(w).T  (see include/qmv.h)."""
+    _need("x", x, 2 * M * K); _need("y", y, 2 * M * N)
+    _need_qmv(N, K, bits, group_size, w=w, scales=scales, biases=biases)
     _check("qmv", lib().qmv(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases),
                             _ptr(y), M, N, K, bits, group_size, _stream(stream)))
 
 
 def qmv_noalloc(x, w, scales, biases, y, M, N, K, bits, group_size, stream=None):
     """qmv without device allocation by the library (see include/qmv.h)."""
+    _need("x", x, 2 * M * K); _need("y", y, 2 * M * N)
+    _need_qmv(N, K, bits, group_size, w=w, scales=scales, biases=biases)
     _check("qmv_noalloc", lib().qmv_noalloc(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases),
                                             _ptr(y), M, N, K, bits, group_size,
                                             _stream(stream)))
 
 
+def qvm(x, w, scales, biases, y, M, K, N, bits, group_size, stream=None):
+    """y[M,N] = x[M,K] @ dequant(w) for w of K rows of N codes (see include/qmv.h)."""
+    _need("x", x, 2 * M * K); _need("y", y, 2 * M * N)
+    _need_qmv(K, N, bits, group_size, w=w, scales=scales, biases=biases)
+    _check("qvm", lib().qvm(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(y),
+                            M, K, N, bits, group_size, _stream(stream)))
+
+
 def qmv_gate_up(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up,
                 M, N, K, bits, group_size, stream=None):
     """y_gate = x @ dequant(w_gate).T and y_up = x @ dequant(w_up).T, one launch."""
+    _need("x", x, 2 * M * K); _need("y_gate", y_gate, 2 * M * N); _need("y_up", y_up, 2 * M * N)
+    _need_qmv(N, K, bits, group_size, w=w_gate, scales=s_gate, biases=b_gate)
+    _need_qmv(N, K, bits, group_size, w=w_up, scales=s_up, biases=b_up)
     _check("qmv_gate_up", lib().qmv_gate_up(
         _ptr(x), _ptr(w_gate), _ptr(s_gate), _ptr(b_gate), _ptr(w_up),
         _ptr(s_up), _ptr(b_up), _ptr(y_gate), _ptr(y_up), M, N, K, bits,
@@ -150,6 +187,9 @@ def qmv_gate_up(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up,
 def qmv_silu_gate_resid(gate, up, x_resid, w, scales, biases, y, M, N, K,
                         bits, group_size, stream=None):
     """y = x_resid + dequant(w) @ (silu(gate) * up); x_resid may be None."""
+    _need("gate", gate, 2 * M * K); _need("up", up, 2 * M * K); _need("y", y, 2 * M * N)
+    _need("x_resid", x_resid, 2 * M * N)
+    _need_qmv(N, K, bits, group_size, w=w, scales=scales, biases=biases)
     _check("qmv_silu_gate_resid", lib().qmv_silu_gate_resid(
         _ptr(gate), _ptr(up), _ptr(x_resid), _ptr(w), _ptr(scales),
         _ptr(biases), _ptr(y), M, N, K, bits, group_size, _stream(stream)))
@@ -159,6 +199,9 @@ def gather_qmv(x, w, scales, biases, lhs_indices, rhs_indices, y, num_pairs,
                num_x_rows, num_experts, N, K, bits, group_size,
                sorted_indices=False, d_status=None, stream=None):
     """y[p] = x[lhs[p]] @ dequant(w[rhs[p]]).T for every pair p."""
+    _need("x", x, 2 * num_x_rows * K); _need("y", y, 2 * num_pairs * N)
+    _need("lhs_indices", lhs_indices, 4 * num_pairs); _need("rhs_indices", rhs_indices, 4 * num_pairs)
+    _need_qmv(num_experts * N, K, bits, group_size, w=w, scales=scales, biases=biases)
     _check("gather_qmv", lib().gather_qmv(
         _ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(lhs_indices),
         _ptr(rhs_indices), _ptr(y), num_pairs, num_x_rows, num_experts, N, K,
@@ -168,6 +211,8 @@ def gather_qmv(x, w, scales, biases, lhs_indices, rhs_indices, y, num_pairs,
 
 def affine_quantize(w, w_q, scales, biases, N, K, bits, group_size, stream=None):
     """Quantize bf16 w[N,K] into packed w_q and bf16 scales/biases [N,K/gs]."""
+    _need("w", w, 2 * N * K)
+    _need_qmv(N, K, bits, group_size, w=w_q, scales=scales, biases=biases)
     _check_quant("affine_quantize", lib().affine_quantize(
         _ptr(w), _ptr(w_q), _ptr(scales), _ptr(biases), N, K, bits, group_size,
         _stream(stream)))
@@ -176,6 +221,8 @@ def affine_quantize(w, w_q, scales, biases, N, K, bits, group_size, stream=None)
 def affine_dequantize(w_q, scales, biases, w_hat, N, K, bits, group_size,
                       stream=None):
     """w_hat[N,K] = bf16(scale * q + bias) from the packed format."""
+    _need("w_hat", w_hat, 2 * N * K)
+    _need_qmv(N, K, bits, group_size, w=w_q, scales=scales, biases=biases)
     _check_quant("affine_dequantize", lib().affine_dequantize(
         _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(w_hat), N, K, bits,
         group_size, _stream(stream)))

@@ -18,6 +18,7 @@
 #include "qmv.h"
 #include "qmv_decode.cuh"
 #include "qmv_mma.cuh"
+#include "qmv_qvm.cuh"
 #include "qmv_stream.cuh"
 
 namespace {
@@ -747,6 +748,30 @@ int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *sca
   return launch(pl, bits, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// qvm (qmv_qvm.cuh)
+// ---------------------------------------------------------------------------
+template <int BITS>
+int launch_qvm_t(const qmvk::QvmParams &p, cudaStream_t stream) {
+  const int nblk = (p.N + qmvk::kQvmCols - 1) / qmvk::kQvmCols;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nblk, qmvk::kQvmCluster, p.M);
+  cfg.blockDim = dim3(qmvk::kQvmWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, qmvk::qvm_kernel<BITS>, p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "qvm launch: %s", cudaGetErrorString(le));
+  }
+  return ok();
+}
+
 }  // namespace
 
 extern "C" {
@@ -778,6 +803,51 @@ int qmv_noalloc(const void *x, const uint32_t *w, const void *scales, const void
                 void *y, int M, int N, int K, int bits, int group_size, void *stream) {
   return qmv_impl("qmv_noalloc", x, w, scales, biases, y, M, N, K, bits, group_size, stream,
                   true);
+}
+
+int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases, void *y,
+        int M, int K, int N, int bits, int group_size, void *stream) {
+  if (!x || !w || !scales || !biases || !y)
+    return fail(QMV_ERR_NULL, "qvm: a buffer pointer is NULL");
+  // W has K rows of N codes; the groups run along N (the output axis)
+  if (!bits_supported(bits))
+    return fail(QMV_ERR_UNSUPPORTED, "qvm: bits=%d not in {2,3,4,5,6,8}", bits);
+  if (!gs_supported(group_size))
+    return fail(QMV_ERR_UNSUPPORTED, "qvm: group_size=%d not in {32,64,128}", group_size);
+  if (K <= 0 || N <= 0) return fail(QMV_ERR_SHAPE, "qvm: K=%d and N=%d must be positive", K, N);
+  if (N % group_size != 0)
+    return fail(QMV_ERR_SHAPE, "qvm: N=%d is not a multiple of group_size=%d", N, group_size);
+  int rc;
+  if (M <= 0) return fail(QMV_ERR_SHAPE, "qvm: M=%d must be positive", M);
+  if (M > 65535) return fail(QMV_ERR_UNSUPPORTED, "qvm: M=%d above 65535", M);
+  const void *ptrs[] = {x, w, scales, biases, y};
+  for (const void *q : ptrs)
+    if (!aligned16(q)) return fail(QMV_ERR_ALIGN, "qvm: buffers must be 16-byte aligned");
+  DeviceInfo *dev;
+  if ((rc = device_info(&dev))) return rc;
+  qmvk::QvmParams p;
+  std::memset(&p, 0, sizeof p);
+  p.w = reinterpret_cast<const uint8_t *>(w);
+  p.s = static_cast<const uint16_t *>(scales);
+  p.b = static_cast<const uint16_t *>(biases);
+  p.x = static_cast<const uint16_t *>(x);
+  p.y = static_cast<uint16_t *>(y);
+  p.M = M;
+  p.K = K;
+  p.N = N;
+  p.G = N / group_size;
+  p.gs_shift = group_size == 32 ? 5 : group_size == 64 ? 6 : 7;
+  p.row_bytes = static_cast<uint32_t>(static_cast<long long>(N) * bits / 8);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (bits) {
+    case 2: return launch_qvm_t<2>(p, st);
+    case 3: return launch_qvm_t<3>(p, st);
+    case 4: return launch_qvm_t<4>(p, st);
+    case 5: return launch_qvm_t<5>(p, st);
+    case 6: return launch_qvm_t<6>(p, st);
+    case 8: return launch_qvm_t<8>(p, st);
+    default: return fail(QMV_ERR_UNSUPPORTED, "qvm: bits=%d", bits);
+  }
 }
 
 int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,

@@ -118,6 +118,17 @@ def workload(name):
                             sorted=srt == "sorted"))
         cfg = {"workload": "MoE gather_qmv", "experts": E, "N": N, "K": K, "bits": bits,
                "group_size": gs, "tokens": T, "top_k": k, "touched_experts": touched}
+    elif name == "qvm":
+        # the non-transposed product over the decode weight shape read the
+        # other way: x [1, 14336] @ dequant(W [14336 rows of 4096 codes])
+        M, K, N, bits, gs = 1, 14336, 4096, 4, 64
+        _, w, s, b = synth.qmv_inputs(1, K, N, bits, gs, seed=7004)
+        x = synth.normal_bf16((M, K), seed=7005)
+        nb = K * N * bits // 8 + 2 * 2 * K * (N // gs) + 2 * M * K + 2 * M * N
+        L.append(Launch(f"qvm_b{bits}", "qvm", nb, M=M, K=K, N=N, bits=bits, gs=gs,
+                        x=x, w=w, s=s, b=b))
+        cfg = {"workload": "qvm (x @ dequant(W))", "M": M, "K": K, "N": N,
+               "group_size": gs, "bits": bits}
     elif name == "quantize":
         # the producer side of the format on the decode weight shape: one
         # quantize of a bf16 matrix and one dequantize of a packed matrix
@@ -149,16 +160,16 @@ def _dev(a, torch):
 
 # Per launch kind: the arrays rotated across weight copies, the per-step
 # inputs (copied from the host in the end-to-end timing) and the outputs.
-_WEIGHTS = {"qmv": ("w", "s", "b"), "gate_up": ("wg", "sg", "bg", "wu", "su", "bu"),
+_WEIGHTS = {"qmv": ("w", "s", "b"), "qvm": ("w", "s", "b"), "gate_up": ("wg", "sg", "bg", "wu", "su", "bu"),
             "silu": ("w", "s", "b"), "gather": ("w", "s", "b"),
             "quantize": ("w",), "dequantize": ("w", "s", "b")}
-_INPUTS = {"qmv": ("x",), "gate_up": ("x",), "silu": ("gate", "up", "resid"),
+_INPUTS = {"qmv": ("x",), "qvm": ("x",), "gate_up": ("x",), "silu": ("gate", "up", "resid"),
            "gather": ("x", "lhs", "rhs"), "quantize": ("w",), "dequantize": ()}
 
 
 def _outputs(l):
     """(name, shape, numpy dtype) of the arrays a launch writes."""
-    if l.kind == "qmv":
+    if l.kind in ("qmv", "qvm"):
         return [("y", (l.M, l.N), np.uint16)]
     if l.kind == "gate_up":
         return [("yg", (l.M, l.N), np.uint16), ("yu", (l.M, l.N), np.uint16)]
@@ -245,6 +256,8 @@ class DeviceWorkload:
         O = {n: self.out.view(j) for n, j in self.out_idx[i].items()}
         if l.kind == "qmv":
             agq.qmv(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.N, l.K, l.bits, l.gs)
+        elif l.kind == "qvm":
+            agq.qvm(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.K, l.N, l.bits, l.gs)
         elif l.kind == "gate_up":
             agq.qmv_gate_up(I["x"], c["wg"], c["sg"], c["bg"], c["wu"], c["su"], c["bu"],
                             O["yg"], O["yu"], l.M, l.N, l.K, l.bits, l.gs)
@@ -598,7 +611,8 @@ def _spawn_replicas(args):
     return subprocess.call(cmd)
 
 
-ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "moe_gather", "quantize")
+ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "moe_gather", "qvm",
+                 "quantize")
 
 
 def run_ours(args):
@@ -647,6 +661,8 @@ def _oracle_launch(l, rows, nthreads):
     elif l.kind == "silu":
         oracle.silu_gate_resid(l.gate, l.up, l.resid, l.w, l.s, l.b, l.M, l.N, l.K, l.bits,
                                l.gs, rows=rows, nthreads=nthreads)
+    elif l.kind == "qvm":
+        oracle.qvm(l.x, l.w, l.s, l.b, l.M, l.K, l.N, l.bits, l.gs)
     elif l.kind == "gather":
         oracle.gather(l.x, l.w, l.s, l.b, l.lhs, l.rhs, l.P, l.T, l.E, l.N, l.K,
                       l.bits, l.gs, nthreads=nthreads)
@@ -669,7 +685,7 @@ def _threads_used(launches, nthreads):
 
 def _sample(l, frac):
     """Rows evaluated per launch and the bytes that sample stands for."""
-    if l.kind == "gather":
+    if l.kind in ("gather", "qvm"):
         return None, l.nbytes
     nr = max(1, int(l.N * frac))
     rows = np.arange(nr, dtype=np.int32)
@@ -705,7 +721,7 @@ def cpu_baseline(launches, budget_s=20.0, frac=None):
             "cores": _threads_used(launches, nthreads),
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"{passes} pass(es) over the first {frac:.3f} of the rows of "
-                      f"every launch of one step (gather: all pairs), plain-C "
+                      f"every launch of one step (gather and qvm: whole), plain-C "
                       f"oracle, {_threads_used(launches, nthreads)} thread(s)"}
 
 

@@ -106,6 +106,26 @@ int qmv_noalloc(const void *x, const uint32_t *w, const void *scales,
                 int group_size, void *stream);
 
 /*
+ * qvm -- y = x @ dequant(W), the non-transposed product
+ *
+ * Defined by the pages' quantized_matmul with transpose = false
+ * ("mlx/include/mlx/backend/metal/kernels/quantized.h": qvm_impl /
+ * affine_qvm, the product the pages use for gradients).  W has K rows of N
+ * codes each, in the packed row format above, and its groups run along N:
+ *   x       bf16 [M, K]
+ *   w       uint32 [K, N*bits/32]
+ *   scales  bf16 [K, N/group_size]
+ *   biases  bf16 [K, N/group_size]
+ *   y       bf16 [M, N]  (written; must not overlap the inputs)
+ *   y[m][n] = sum_k x[m][k] * (scale[k][n/gs] * q[k][n] + bias[k][n/gs])
+ * N a positive multiple of group_size, K >= 1, 1 <= M <= 65535.  The rows
+ * are split between the CTAs of a thread-block cluster whose partial sums
+ * are added in a fixed order (deterministic results, no scratch memory).
+ */
+int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases, void *y,
+        int M, int K, int N, int bits, int group_size, void *stream);
+
+/*
  * qmv_gate_up -- dual-output GEMV over one input, in ONE kernel launch:
  *   y_gate = x @ dequant(W_gate).T,   y_up = x @ dequant(W_up).T
  *

@@ -178,3 +178,24 @@ def test_quant_binding_raises_with_its_own_message(lib):
     with pytest.raises(agq.QmvError) as ei:
         agq.affine_dequantize(A, A, A, A, 2, 128, 9, 64, stream=0)
     assert ei.value.status == agq.QMV_ERR_UNSUPPORTED and "bits=9" in str(ei.value)
+
+
+def test_qvm_argument_checks(lib):
+    q = lib.qvm
+    P = ctypes.c_void_p
+    q.argtypes = [P, P, P, P, P] + [ctypes.c_int] * 5 + [P]
+    ok = [A, A, A, A, A, 1, 128, 256, 4, 64, None]
+
+    def call(i=None, v=None):
+        args = list(ok)
+        if i is not None:
+            args[i] = v
+        return q(*args)
+
+    assert call(0, None) == agq.QMV_ERR_NULL
+    assert call(8, 7) == agq.QMV_ERR_UNSUPPORTED          # bits
+    assert call(9, 48) == agq.QMV_ERR_UNSUPPORTED         # group size
+    assert call(7, 200) == agq.QMV_ERR_SHAPE              # N % gs
+    assert call(5, 0) == agq.QMV_ERR_SHAPE                # M
+    assert call(6, 0) == agq.QMV_ERR_SHAPE                # K
+    assert call(1, A + 4) == agq.QMV_ERR_ALIGN

@@ -212,3 +212,10 @@ def test_every_workload_has_inputs_outputs_and_weights(name):
             assert getattr(l, k) is not None, (l.label, k)
         outs = bench._outputs(l)
         assert outs and all(int(np.prod(s)) > 0 for _, s, _ in outs)
+
+
+def test_qvm_workload_arrays_have_the_launch_shapes():
+    (l,), _ = bench.workload("qvm")
+    assert l.x.shape == (l.M, l.K)
+    assert l.w.shape == (l.K, l.N * l.bits // 32) and l.s.shape == (l.K, l.N // l.gs)
+    assert l.nbytes == _arrays_bytes(l.w, l.s, l.b, l.x) + 2 * l.M * l.N
