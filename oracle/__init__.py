@@ -50,6 +50,11 @@ def lib() -> ctypes.CDLL:
         L.oracle_dequantize_bf16.argtypes = [P, P, P, I, I, I, I, P]
         L.oracle_affine_quantize.argtypes = [P, I, I, I, I, P, P, P]
         L.oracle_qvm.argtypes = [P, P, P, P, I, I, I, I, I, P, P]
+        L.oracle_trellis_value.restype = ctypes.c_double
+        L.oracle_trellis_value.argtypes = [ctypes.c_uint32]
+        L.oracle_trellis_state.restype = ctypes.c_uint32
+        L.oracle_trellis_state.argtypes = [ctypes.c_uint32, ctypes.c_uint32, I, I]
+        L.oracle_qmv_trellis.argtypes = [P, P, P, I, I, I, I, P, P]
         _lib = L
     return _lib
 
@@ -190,4 +195,24 @@ def qvm(x, w, scales, biases, M, K, N, bits, gs):
     y = np.zeros((M, N)); a = np.zeros((M, N))
     if lib().oracle_qvm(_p(x), _p(w), _p(s), _p(b), M, K, N, bits, gs, _p(y), _p(a)):
         raise ValueError("oracle_qvm: bad arguments")
+    return y, a
+
+
+def trellis_value(state: int) -> float:
+    """Value of a 16-bit trellis state (the pages' inst3)."""
+    return lib().oracle_trellis_value(int(state))
+
+
+def trellis_state(w0: int, w1: int, t: int, bits: int) -> int:
+    """State of value t of word w0 with successor word w1."""
+    return int(lib().oracle_trellis_state(int(w0), int(w1), int(t), int(bits)))
+
+
+def qmv_trellis(x, w, scales, M, N, K, bits):
+    """Trellis-mode y[M, N] = scale * x @ V.T (scale = scales[0]); returns
+    (y, a) with a = |scale| * sum_k |x * v|."""
+    x, w, s = _c(x, np.uint16), _c(w, np.uint32), _c(scales, np.uint16)
+    y = np.zeros((M, N)); a = np.zeros((M, N))
+    if lib().oracle_qmv_trellis(_p(x), _p(w), _p(s), M, N, K, bits, _p(y), _p(a)):
+        raise ValueError("oracle_qmv_trellis: bad arguments")
     return y, a

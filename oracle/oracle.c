@@ -556,3 +556,106 @@ int oracle_qvm(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Trellis mode ("Get trellis to run" compare page, quantized.h: inst3 and   */
+/* qmv_trellis_impl)                                                         */
+/* ------------------------------------------------------------------------ */
+
+/* IEEE binary16 bit pattern -> double (exact). */
+static double f16_to_double(uint16_t h)
+{
+    const int sign = h >> 15, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);                 /* subnormal */
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + m), e - 25);            /* (1 + m/1024) 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* The binary16 value nearest to v (ties to even), as a double.  v is the
+ * exact sum of two binary16 values, so it is exact in double. */
+static double round_to_f16(double v)
+{
+    if (v == 0.0 || isnan(v) || isinf(v)) return v;
+    int e;
+    frexp(fabs(v), &e);                /* 2^(e-1) <= |v| < 2^e */
+    int ulp_exp = e - 11;              /* 11 significant bits */
+    if (ulp_exp < -24) ulp_exp = -24;  /* subnormal spacing */
+    const double n = nearbyint(ldexp(v, -ulp_exp));  /* default mode: ties to even */
+    const double r = ldexp(n, ulp_exp);
+    if (fabs(r) > 65504.0) return v > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
+/* The value of a 16-bit trellis state (the page's inst3 with its default
+ * constants a = 89226354, b = 64248484, m = 996162400): x = a * state + b in
+ * 32-bit unsigned arithmetic, keep the sign bit and the low 12 bits of each
+ * 16-bit half (mask 0x8FFF8FFF), XOR m, read the two halves as binary16
+ * numbers and add them in binary16.
+ * Pins: every state against an independent numpy float16 computation; a
+ * hand-worked state (tests/golden/trellis.txt); the range of all values. */
+double oracle_trellis_value(uint32_t state)
+{
+    uint32_t x = 89226354u * (state & 0xFFFFu) + 64248484u;
+    x = (x & 0x8FFF8FFFu) ^ 996162400u;
+    return round_to_f16(f16_to_double((uint16_t)(x & 0xFFFFu)) +
+                        f16_to_double((uint16_t)(x >> 16)));
+}
+
+/* The state of value t (0 <= t < 16/bits) of word w0, whose successor word
+ * is w1 (qmv_trellis_impl): t = 0 reads w0 itself; value t >= 1 takes its
+ * low bits * t bits from w1 -- w0 ^ ((w0 ^ w1) & (2^(bits*t) - 1)) -- with
+ * bit 0 of that part flipped for odd t, and bit `bits` flipped for t = 1.
+ * Pins: the page's eight (2-bit) and four (4-bit) printed expressions, on
+ * random word pairs. */
+uint32_t oracle_trellis_state(uint32_t w0, uint32_t w1, int t, int bits)
+{
+    w0 &= 0xFFFFu;
+    w1 &= 0xFFFFu;
+    if (t == 0) return w0;
+    const uint32_t wx = (w0 ^ w1) ^ ((t & 1) ? 1u : 0u);
+    uint32_t s = w0 ^ (wx & ((1u << (bits * t)) - 1u));
+    if (t == 1) s ^= 1u << bits;
+    return s & 0xFFFFu;
+}
+
+/* Trellis-mode GEMV: y[m][n] = scale * sum_k x[m][k] * v(n, k), with scale
+ * the first element of `scales` (the page's kernel reads scales[0]; biases
+ * are not used), and a[m][n] = |scale| * sum_k |x[m][k] * v(n, k)|.
+ * Row n is W = K*bits/16 little-endian 16-bit words u_0 .. u_{W-1}; value
+ * k = i * (16/bits) + t has state oracle_trellis_state(u_i, u_{(i+1) mod W},
+ * t, bits): the successor of the row's last word is its first word (the
+ * reading of the page's successor word; see the design notes).
+ * bits in {2, 4}; K * bits a multiple of 32 (rows of whole uint32 words).
+ * Pins: a dense fp64 matmul of the value matrix built by the test's own
+ * decoder; brute force on a tiny matrix with dyadic x. */
+int oracle_qmv_trellis(const uint16_t *x, const uint32_t *w, const uint16_t *scales, int M,
+                       int N, int K, int bits, double *y, double *a)
+{
+    if (M < 0 || N < 0 || K <= 0 || !(bits == 2 || bits == 4) || (K * bits) % 32 != 0)
+        return -1;
+    const long long W = (long long)K * bits / 16;
+    const int cpw = 16 / bits;
+    const double scale = oracle_bf16_to_double(scales[0]);
+    for (long long n = 0; n < N; ++n) {
+        const uint8_t *row = (const uint8_t *)w + n * W * 2;
+        for (long long m = 0; m < M; ++m) {
+            double acc = 0.0, mag = 0.0;
+            for (long long i = 0; i < W; ++i) {
+                const long long j = (i + 1) % W;
+                const uint32_t w0 = row[2 * i] | ((uint32_t)row[2 * i + 1] << 8);
+                const uint32_t w1 = row[2 * j] | ((uint32_t)row[2 * j + 1] << 8);
+                for (int t = 0; t < cpw; ++t) {
+                    const double v = oracle_trellis_value(oracle_trellis_state(w0, w1, t, bits));
+                    const double p = oracle_bf16_to_double(x[m * K + i * cpw + t]) * v;
+                    acc += p;
+                    mag += fabs(p);
+                }
+            }
+            y[m * N + n] = scale * acc;
+            a[m * N + n] = fabs(scale) * mag;
+        }
+    }
+    return 0;
+}

@@ -44,4 +44,8 @@ int oracle_affine_quantize(const uint16_t *w, int N, int K, int bits, int gs,
 int oracle_qvm(const uint16_t *x, const uint32_t *w, const uint16_t *scales,
                const uint16_t *biases, int M, int K, int N, int bits, int gs,
                double *y, double *a);
+double oracle_trellis_value(uint32_t state);
+uint32_t oracle_trellis_state(uint32_t w0, uint32_t w1, int t, int bits);
+int oracle_qmv_trellis(const uint16_t *x, const uint32_t *w, const uint16_t *scales, int M,
+                       int N, int K, int bits, double *y, double *a);
 #endif
