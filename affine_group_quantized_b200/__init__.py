@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.qmv_abi_version.restype = I
         L.qmv_abi_version.argtypes = []
         L.qvm.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+        L.qmv_trellis.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.qmv_trellis.restype = I
         L.qvm.restype = I
         L.qmv_device_status.argtypes = [P, I, P]
         L.qmv_device_status.restype = I
@@ -78,7 +80,7 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-EXPORTED = ("qmv", "qmv_noalloc", "qvm", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
+EXPORTED = ("qmv", "qmv_noalloc", "qvm", "qmv_trellis", "qmv_gate_up", "qmv_silu_gate_resid", "gather_qmv",
             "qmv_last_error", "qmv_abi_version", "qmv_device_status", "affine_quantize",
             "affine_dequantize", "qmv_quant_last_error")
 
@@ -170,6 +172,14 @@ def qvm(x, w, scales, biases, y, M, K, N, bits, group_size, stream=None):
     _need_qmv(K, N, bits, group_size, w=w, scales=scales, biases=biases)
     _check("qvm", lib().qvm(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(y),
                             M, K, N, bits, group_size, _stream(stream)))
+
+
+def qmv_trellis(x, w, scales, y, M, N, K, bits, stream=None):
+    """Trellis-mode y[M,N] = scales[0] * x @ V.T (see include/qmv.h)."""
+    _need("x", x, 2 * M * K); _need("y", y, 2 * M * N)
+    _need("w", w, N * K * bits // 8); _need("scales", scales, 2)
+    _check("qmv_trellis", lib().qmv_trellis(_ptr(x), _ptr(w), _ptr(scales), _ptr(y),
+                                            M, N, K, bits, _stream(stream)))
 
 
 def qmv_gate_up(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, y_gate, y_up,

@@ -20,6 +20,7 @@
 #include "qmv_mma.cuh"
 #include "qmv_qvm.cuh"
 #include "qmv_stream.cuh"
+#include "qmv_trellis.cuh"
 
 namespace {
 
@@ -772,6 +773,43 @@ int launch_qvm_t(const qmvk::QvmParams &p, cudaStream_t stream) {
   return ok();
 }
 
+// ---------------------------------------------------------------------------
+// Trellis mode (qmv_trellis.cuh)
+// ---------------------------------------------------------------------------
+template <int BITS>
+int launch_trellis_t(const qmvk::TrellisParams &p, int sms, cudaStream_t stream) {
+  auto kern = qmvk::qmv_trellis_kernel<BITS>;
+  const int smem = 4 * p.K;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int granted[kMaxDevices] = {};
+  if (smem > 48 * 1024 && smem > granted[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    granted[dev] = smem;
+  }
+  const int rows_per_cta = qmvk::kTrellisWarps;
+  long long grid = (p.N + rows_per_cta - 1) / rows_per_cta;
+  if (grid > 16LL * sms) grid = 16LL * sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), p.M);
+  cfg.blockDim = dim3(qmvk::kTrellisWarps * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "qmv_trellis launch: %s", cudaGetErrorString(le));
+  }
+  return ok();
+}
+
 }  // namespace
 
 extern "C" {
@@ -848,6 +886,42 @@ int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases
     case 8: return launch_qvm_t<8>(p, st);
     default: return fail(QMV_ERR_UNSUPPORTED, "qvm: bits=%d", bits);
   }
+}
+
+int qmv_trellis(const void *x, const uint32_t *w, const void *scales, void *y, int M, int N,
+                int K, int bits, void *stream) {
+  if (!x || !w || !scales || !y)
+    return fail(QMV_ERR_NULL, "qmv_trellis: a buffer pointer is NULL");
+  if (bits != 2 && bits != 4)
+    return fail(QMV_ERR_UNSUPPORTED, "qmv_trellis: bits=%d not in {2,4}", bits);
+  if (M <= 0 || N <= 0 || K <= 0)
+    return fail(QMV_ERR_SHAPE, "qmv_trellis: M=%d, N=%d, K=%d must be positive", M, N, K);
+  if ((static_cast<long long>(K) * bits) % 128 != 0)
+    return fail(QMV_ERR_SHAPE, "qmv_trellis: K*bits=%lld is not a multiple of 128",
+                static_cast<long long>(K) * bits);
+  if (K > 49152) return fail(QMV_ERR_UNSUPPORTED, "qmv_trellis: K=%d above 49152", K);
+  if (M > 65535) return fail(QMV_ERR_UNSUPPORTED, "qmv_trellis: M=%d above 65535", M);
+  const void *ptrs[] = {x, w, y};
+  for (const void *q : ptrs)
+    if (!aligned16(q))
+      return fail(QMV_ERR_ALIGN, "qmv_trellis: buffers must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(scales) & 1u)
+    return fail(QMV_ERR_ALIGN, "qmv_trellis: scales must be 2-byte aligned");
+  DeviceInfo *dev;
+  int rc;
+  if ((rc = device_info(&dev))) return rc;
+  qmvk::TrellisParams p;
+  std::memset(&p, 0, sizeof p);
+  p.w = reinterpret_cast<const uint16_t *>(w);
+  p.x = static_cast<const uint16_t *>(x);
+  p.scales = static_cast<const uint16_t *>(scales);
+  p.y = static_cast<uint16_t *>(y);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.W = static_cast<int>(static_cast<long long>(K) * bits / 16);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return bits == 2 ? launch_trellis_t<2>(p, dev->sms, st) : launch_trellis_t<4>(p, dev->sms, st);
 }
 
 int qmv_gate_up(const void *x, const uint32_t *w_gate, const void *s_gate,

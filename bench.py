@@ -25,6 +25,7 @@ import threading
 import time
 
 import numpy as np
+import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -129,6 +130,18 @@ def workload(name):
                         x=x, w=w, s=s, b=b))
         cfg = {"workload": "qvm (x @ dequant(W))", "M": M, "K": K, "N": N,
                "group_size": gs, "bits": bits}
+    elif name == "trellis":
+        # the trellis-mode decode GEMV on the decode shape, 2- and 4-bit
+        M, N, K = 1, 14336, 4096
+        for bits in (2, 4):
+            rng = np.random.default_rng(8100 + bits)
+            w = rng.integers(0, 1 << 32, size=(N, K * bits // 32), dtype=np.uint64).astype(np.uint32)
+            x = synth.normal_bf16((M, K), seed=8110 + bits)
+            s = synth.bf16_bits(torch.tensor([0.0123]))
+            nb = N * K * bits // 8 + 2 + 2 * M * K + 2 * M * N
+            L.append(Launch(f"trellis_b{bits}", "trellis", nb, M=M, N=N, K=K, bits=bits, gs=0,
+                            x=x, w=w, s=s))
+        cfg = {"workload": "trellis-mode decode GEMV", "M": M, "K": K, "N": N, "bits": [2, 4]}
     elif name == "quantize":
         # the producer side of the format on the decode weight shape: one
         # quantize of a bf16 matrix and one dequantize of a packed matrix
@@ -160,16 +173,16 @@ def _dev(a, torch):
 
 # Per launch kind: the arrays rotated across weight copies, the per-step
 # inputs (copied from the host in the end-to-end timing) and the outputs.
-_WEIGHTS = {"qmv": ("w", "s", "b"), "qvm": ("w", "s", "b"), "gate_up": ("wg", "sg", "bg", "wu", "su", "bu"),
+_WEIGHTS = {"qmv": ("w", "s", "b"), "qvm": ("w", "s", "b"), "trellis": ("w", "s"), "gate_up": ("wg", "sg", "bg", "wu", "su", "bu"),
             "silu": ("w", "s", "b"), "gather": ("w", "s", "b"),
             "quantize": ("w",), "dequantize": ("w", "s", "b")}
-_INPUTS = {"qmv": ("x",), "qvm": ("x",), "gate_up": ("x",), "silu": ("gate", "up", "resid"),
+_INPUTS = {"qmv": ("x",), "qvm": ("x",), "trellis": ("x",), "gate_up": ("x",), "silu": ("gate", "up", "resid"),
            "gather": ("x", "lhs", "rhs"), "quantize": ("w",), "dequantize": ()}
 
 
 def _outputs(l):
     """(name, shape, numpy dtype) of the arrays a launch writes."""
-    if l.kind in ("qmv", "qvm"):
+    if l.kind in ("qmv", "qvm", "trellis"):
         return [("y", (l.M, l.N), np.uint16)]
     if l.kind == "gate_up":
         return [("yg", (l.M, l.N), np.uint16), ("yu", (l.M, l.N), np.uint16)]
@@ -256,6 +269,8 @@ class DeviceWorkload:
         O = {n: self.out.view(j) for n, j in self.out_idx[i].items()}
         if l.kind == "qmv":
             agq.qmv(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.N, l.K, l.bits, l.gs)
+        elif l.kind == "trellis":
+            agq.qmv_trellis(I["x"], c["w"], c["s"], O["y"], l.M, l.N, l.K, l.bits)
         elif l.kind == "qvm":
             agq.qvm(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.K, l.N, l.bits, l.gs)
         elif l.kind == "gate_up":
@@ -612,7 +627,7 @@ def _spawn_replicas(args):
 
 
 ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "moe_gather", "qvm",
-                 "quantize")
+                 "trellis", "quantize")
 
 
 def run_ours(args):
@@ -663,6 +678,9 @@ def _oracle_launch(l, rows, nthreads):
                                l.gs, rows=rows, nthreads=nthreads)
     elif l.kind == "qvm":
         oracle.qvm(l.x, l.w, l.s, l.b, l.M, l.K, l.N, l.bits, l.gs)
+    elif l.kind == "trellis":
+        n = l.N if rows is None else len(rows)
+        oracle.qmv_trellis(l.x, l.w[:n], l.s, l.M, n, l.K, l.bits)
     elif l.kind == "gather":
         oracle.gather(l.x, l.w, l.s, l.b, l.lhs, l.rhs, l.P, l.T, l.E, l.N, l.K,
                       l.bits, l.gs, nthreads=nthreads)

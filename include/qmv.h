@@ -126,6 +126,28 @@ int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases
         int M, int K, int N, int bits, int group_size, void *stream);
 
 /*
+ * qmv_trellis -- trellis-mode GEMV: y = scale * x @ V.T
+ *
+ * Defined by the pages' trellis decode ("Get trellis to run" compare page,
+ * quantized.h: inst3 and qmv_trellis_impl).  Row n of W is K*bits/16
+ * little-endian 16-bit words (the packed row bytes read as uint16).  Value k
+ * = i*(16/bits) + t of the row has a 16-bit state built from word i and its
+ * successor word (word i+1; the row's last word is followed by its first):
+ * t = 0 reads word i; t >= 1 takes the low bits*t bits from the successor,
+ * with bit 0 of that part flipped for odd t and bit `bits` flipped for t = 1.
+ * v(n, k) = inst3(state): x = 89226354*state + 64248484 (32-bit), keep the
+ * sign and low 12 bits of each 16-bit half, XOR 996162400, and add the two
+ * halves as binary16 numbers (one binary16 rounding).
+ *   x       bf16 [M, K]
+ *   w       uint32 [N, K*bits/32]
+ *   scales  bf16; scales[0] scales the whole matrix (no groups, no biases)
+ *   y       bf16 [M, N]  = bf16(scales[0] * sum_k x[m][k] * v(n, k)), fp32 sums
+ * bits in {2, 4}; K*bits a multiple of 128, K <= 49152; 1 <= M <= 65535.
+ */
+int qmv_trellis(const void *x, const uint32_t *w, const void *scales, void *y, int M, int N,
+                int K, int bits, void *stream);
+
+/*
  * qmv_gate_up -- dual-output GEMV over one input, in ONE kernel launch:
  *   y_gate = x @ dequant(W_gate).T,   y_up = x @ dequant(W_up).T
  *

@@ -199,3 +199,23 @@ def test_qvm_argument_checks(lib):
     assert call(5, 0) == agq.QMV_ERR_SHAPE                # M
     assert call(6, 0) == agq.QMV_ERR_SHAPE                # K
     assert call(1, A + 4) == agq.QMV_ERR_ALIGN
+
+
+def test_trellis_argument_checks(lib):
+    q = lib.qmv_trellis
+    P = ctypes.c_void_p
+    q.argtypes = [P, P, P, P] + [ctypes.c_int] * 4 + [P]
+    ok = [A, A, A, A, 1, 8, 256, 4, None]
+
+    def call(i=None, v=None):
+        args = list(ok)
+        if i is not None:
+            args[i] = v
+        return q(*args)
+
+    assert call(2, None) == agq.QMV_ERR_NULL
+    assert call(7, 3) == agq.QMV_ERR_UNSUPPORTED          # bits
+    assert call(6, 40) == agq.QMV_ERR_SHAPE               # K * bits % 128
+    assert call(4, 0) == agq.QMV_ERR_SHAPE                # M
+    assert call(0, A + 2) == agq.QMV_ERR_ALIGN
+    assert call(2, A + 1) == agq.QMV_ERR_ALIGN             # scales need 2 bytes
