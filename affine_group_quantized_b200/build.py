@@ -14,14 +14,14 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libqmv.so")
-SOURCES = ["qmv_api.cu", "qmv_quant.cu"]
+SOURCES = ["qmv_api.cu", "qmv_quant.cu", "qmv_qmm.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "--expt-relaxed-constexpr",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "-Xptxas", "-warn-spills",
 ]
 
@@ -37,11 +37,24 @@ def build(force: bool = False, verbose: bool = False) -> str:
         newest = max(os.path.getmtime(f) for f in _inputs())
         if os.path.getmtime(LIB) >= newest:
             return LIB
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    subprocess.run(cmd, check=True)
+    # one object per source, compiled side by side, then one link
+    objdir = os.path.join(HERE, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    procs, objs = [], []
+    for src in SOURCES:
+        obj = os.path.join(objdir, src.replace(".cu", ".o"))
+        cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj,
+               os.path.join(CSRC, src)]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+    failed = [src for src, pr in procs if pr.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc " + " ".join(failed))
+    link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+            "-o", LIB + ".tmp", *objs]
+    subprocess.run(link, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

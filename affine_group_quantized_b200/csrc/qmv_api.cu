@@ -18,6 +18,7 @@
 #include "qmv.h"
 #include "qmv_decode.cuh"
 #include "qmv_mma.cuh"
+#include "qmv_qmm.h"
 #include "qmv_qvm.cuh"
 #include "qmv_stream.cuh"
 #include "qmv_trellis.cuh"
@@ -100,6 +101,11 @@ constexpr int kMaxDevices = 64;
 #endif
 // fewest activation rows that go to the tensor-core path
 constexpr int kMmaMinRows = QMV_MMA_MIN_ROWS;
+#ifndef QMV_QMM_MIN_ROWS
+#define QMV_QMM_MIN_ROWS 17
+#endif
+// fewest activation rows that go to the many-row tensor-core kernel
+constexpr int kQmmMinRows = QMV_QMM_MIN_ROWS;
 DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 
@@ -482,8 +488,8 @@ void init_decode(DecodePlan &dp, const void *x, int N, int K, int nmat, const De
 bool mma_path(int M, int K, int bits, int gs) {
   if (!(bits == 2 || bits == 4 || bits == 8)) return false;
   if (!(gs == 32 || gs == 64 || gs == 128)) return false;
-  return M >= kMmaMinRows && M <= qmvk::kMmaCols && K % (1024 / bits) == 0 &&
-         (K / gs) % 8 == 0;
+  return M >= kMmaMinRows && M <= qmvk::kMmaCols && M < kQmmMinRows &&
+         K % (1024 / bits) == 0 && (K / gs) % 8 == 0;
 }
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no link to
@@ -526,19 +532,25 @@ int encode_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, uint6
 // it).  Calls that use it on one device are expected in stream order.
 struct MmaScratch {
   float *part = nullptr;
+  size_t part_bytes = 0;
   int *cnt = nullptr;
   int cnt_len = 0;
 };
 MmaScratch g_mma_scratch[kMaxDevices];
 std::mutex g_mma_scratch_mu;
 
-int mma_scratch(int dev_id, int sms, int ntiles, cudaStream_t stream, MmaScratch **out) {
+int mma_scratch(int dev_id, size_t part_bytes, int ntiles, cudaStream_t stream,
+                MmaScratch **out) {
   std::lock_guard<std::mutex> lock(g_mma_scratch_mu);
   MmaScratch &s = g_mma_scratch[dev_id];
-  if (!s.part) {
-    const size_t bytes = static_cast<size_t>(sms) * 2 * qmvk::kMmaCols * qmvk::kMmaRows * 4;
-    if (cudaMalloc(&s.part, bytes) != cudaSuccess)
-      return fail(QMV_ERR_CUDA, "tensor-core path: cannot allocate %zu bytes of scratch", bytes);
+  if (s.part_bytes < part_bytes) {
+    float *np = nullptr;
+    if (cudaMalloc(&np, part_bytes) != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "tensor-core path: cannot allocate %zu bytes of scratch",
+                  part_bytes);
+    if (s.part) cudaFree(s.part);  // waits for the launches that use it
+    s.part = np;
+    s.part_bytes = part_bytes;
   }
   if (s.cnt_len < ntiles) {
     int n = s.cnt_len ? s.cnt_len : 1024;
@@ -691,7 +703,10 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
   MmaScratch *sc = nullptr;
   int rc;
   if ((rc = fixed_scratch ? static_scratch(d, dev->sms, mp.ntiles, &sc)
-                         : mma_scratch(d, dev->sms, mp.ntiles, stream, &sc)))
+                         : mma_scratch(d,
+                                       static_cast<size_t>(dev->sms) * 2 * qmvk::kMmaCols *
+                                           qmvk::kMmaRows * sizeof(float),
+                                       mp.ntiles, stream, &sc)))
     return rc;
   mp.part = sc->part;
   mp.cnt = sc->cnt;
@@ -702,6 +717,59 @@ int launch_mma(const void *x, const uint32_t *w, const void *scales,
     case 8: return launch_mma_b<8>(mp, gs, grid, dev, stream);
     default: return fail(QMV_ERR_UNSUPPORTED, "bits=%d on the tensor-core path", bits);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Many activation rows (M > 16) on the tensor cores (qmv_qmm.cu): bf16
+// operands, x straight from memory; the same code widths and shape rules as
+// the few-row path.
+// ---------------------------------------------------------------------------
+constexpr long long kQmmMaxTiles = 1LL << 24;
+
+bool qmm_path(int M, int N, int K, int bits, int gs) {
+  if (!(bits == 2 || bits == 4 || bits == 8)) return false;
+  if (!(gs == 32 || gs == 64 || gs == 128)) return false;
+  return M >= kQmmMinRows && M >= kMmaMinRows && K % qmvq::qmm_stage_codes(bits) == 0 &&
+         (K / gs) % 8 == 0 && qmvq::qmm_tiles(M, N) <= kQmmMaxTiles;
+}
+
+int launch_qmm(const void *x, const uint32_t *w, const void *scales, const void *biases,
+               void *y, int M, int N, int K, int bits, int gs, DeviceInfo *dev,
+               cudaStream_t stream, bool fixed_scratch) {
+  qmvq::QmmArgs a;
+  a.x = x;
+  a.w = w;
+  a.scales = scales;
+  a.biases = biases;
+  a.y = y;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.bits = bits;
+  a.gs = gs;
+  a.sms = dev->sms;
+  a.smem_optin = dev->smem_optin;
+  a.err = dev->status;
+  a.part = nullptr;
+  a.cnt = nullptr;
+  a.stream = stream;
+  if (!fixed_scratch) {
+    // split tiles need the partial-sum slots and tile counters; without
+    // scratch (qmv_noalloc) every CTA takes whole tiles
+    int d = 0;
+    cudaGetDevice(&d);
+    MmaScratch *sc = nullptr;
+    int rc;
+    if ((rc = mma_scratch(d, qmvq::qmm_part_bytes(M, dev->sms),
+                          static_cast<int>(qmvq::qmm_tiles(M, N)), stream, &sc)))
+      return rc;
+    a.part = sc->part;
+    a.cnt = sc->cnt;
+  }
+  char msg[256];
+  const int rc = qmvq::qmm_launch(a, msg, sizeof msg);
+  if (rc) return fail(rc, "%s", msg);
+  return ok();
 }
 
 int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *scales,
@@ -719,6 +787,9 @@ int qmv_impl(const char *name, const void *x, const uint32_t *w, const void *sca
   if ((rc = device_info(&dev))) return rc;
   if (mma_path(M, K, bits, group_size))
     return launch_mma(x, w, scales, biases, y, M, N, K, bits, group_size, dev,
+                      static_cast<cudaStream_t>(stream), fixed_scratch);
+  if (qmm_path(M, N, K, bits, group_size))
+    return launch_qmm(x, w, scales, biases, y, M, N, K, bits, group_size, dev,
                       static_cast<cudaStream_t>(stream), fixed_scratch);
   if (decode_path(M, K, bits)) {
     DecodePlan dp;

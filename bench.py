@@ -7,7 +7,7 @@ of the six bit widths (six kernel launches).  Metric: achieved HBM GB/s over
 the step, with algorithmic bytes = packed W + scales + biases + x + y.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_sweep|qmv_small|ffn_int8|batched|moe_gather]
+                    [--workload decode_sweep|qmv_small|ffn_int8|batched|prefill|moe_gather|...]
 
 Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs the
 same workload on its own GPU (independent replicas, no collective on the data
@@ -103,6 +103,18 @@ def workload(name):
                 L.append(Launch(f"qmv_M{M}_gs{gs}", "qmv", qmv_bytes(M, N, K, bits, gs),
                                 M=M, N=N, K=K, bits=bits, gs=gs, x=x, w=w, s=s, b=b))
         cfg = {"workload": "batched decode qmv", "M": [1, 2, 4, 8], "K": K, "N": N,
+               "group_size": [32, 128], "bits": bits}
+    elif name == "prefill":
+        # many activation rows (the pages' qmm_t) on the batched matrix: the
+        # tensor-core contraction; M=32 is memory bound, M=128 tensor bound
+        N, K, bits = 28672, 8192, 4
+        for gs in (32, 128):
+            for M in (32, 128):
+                x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=4500 + M + gs)
+                L.append(Launch(f"qmm_M{M}_gs{gs}", "qmv", qmv_bytes(M, N, K, bits, gs),
+                                M=M, N=N, K=K, bits=bits, gs=gs, x=x, w=w, s=s, b=b,
+                                flops=2 * M * N * K))
+        cfg = {"workload": "prefill qmm", "M": [32, 128], "K": K, "N": N,
                "group_size": [32, 128], "bits": bits}
     elif name == "moe_gather":
         E, N, K, bits, gs, T, k = 64, 1536, 2048, 4, 64, 32, 4
@@ -387,6 +399,16 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def recorded_traffic(kernel_label, workload_name):
     """DRAM bytes per launch from a committed ncu summary, if the kernel
     source has not changed since it was captured."""
@@ -564,6 +586,12 @@ def measure_workload(name, args, torch, world, with_cpu):
             "us_isolated": round(iso * 1e3, 3), "us_basis": basis, "GB/s": round(gbs, 1),
             "frac_of_measured_peak": round(gbs / peak, 4), "bytes": l.nbytes,
             "ncu_us": recorded_ncu_time(l.label, name)}
+    tpeak, tpeak_kind = measured_tensor_peak()
+    for l, d in zip(launches, us_of):
+        if getattr(l, "flops", None):
+            tfs = l.flops / (d * 1e-3) / 1e12
+            out_launch[l.label]["TFLOP/s"] = round(tfs, 1)
+            out_launch[l.label]["frac_of_measured_tensor_peak"] = round(tfs / tpeak, 4)
     dom = max(range(len(launches)), key=lambda i: us_of[i])
     ach = launches[dom].nbytes / (us_of[dom] * 1e-3) / 1e9
     value = job_gbs(world, step_bytes, K, ms)
@@ -584,12 +612,8 @@ def measure_workload(name, args, torch, world, with_cpu):
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        graphs=f"timed steps replayed as CUDA graphs of {copies} steps (one "
                               f"weight rotation); the remainder one step per graph"),
-        "roofline": {"bound": "hbm", "kernel": launches[dom].label,
-                     "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(ach / peak, 4), "peak_kind": peak_kind,
-                     "timing": basis,
-                     "traffic": recorded_traffic(launches[dom].label, name),
-                     "algorithmic_bytes_per_launch": launches[dom].nbytes},
+        "roofline": _roofline(launches[dom], us_of[dom], peak, peak_kind, tpeak, tpeak_kind,
+                              basis, recorded_traffic(launches[dom].label, name)),
         "per_launch": out_launch,
         "tokens_per_s_equiv": {l.label: round(1e6 / (d * 1e3), 1)
                                for l, d in zip(launches, us_of)},
@@ -610,6 +634,24 @@ def measure_workload(name, args, torch, world, with_cpu):
     return res
 
 
+def _roofline(l, ms, peak, peak_kind, tpeak, tpeak_kind, basis, traffic):
+    """The bound of launch l: HBM bytes, or tensor FLOPs where the launch
+    carries them and their time at the measured tensor peak is the longer."""
+    t_mem = l.nbytes / (peak * 1e9)
+    flops = getattr(l, "flops", None)
+    if flops and flops / (tpeak * 1e12) > t_mem:
+        ach = flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "kernel": l.label, "achieved": round(ach, 1),
+                "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
+                "peak_kind": tpeak_kind, "timing": basis, "traffic": traffic,
+                "algorithmic_flops_per_launch": flops,
+                "algorithmic_bytes_per_launch": l.nbytes}
+    ach = l.nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": l.label, "achieved": round(ach, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(ach / peak, 4), "peak_kind": peak_kind,
+            "timing": basis, "traffic": traffic, "algorithmic_bytes_per_launch": l.nbytes}
+
+
 def _spawn_replicas(args):
     """`--gpus N` without torchrun: relaunch this command under torchrun, one
     process per GPU, or stop with an error when fewer GPUs are visible."""
@@ -626,8 +668,8 @@ def _spawn_replicas(args):
     return subprocess.call(cmd)
 
 
-ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "moe_gather", "qvm",
-                 "trellis", "quantize")
+ALL_WORKLOADS = ("decode_sweep", "qmv_small", "ffn_int8", "batched", "prefill", "moe_gather",
+                 "qvm", "trellis", "quantize")
 
 
 def run_ours(args):

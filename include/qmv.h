@@ -77,13 +77,19 @@ typedef enum {
  *   y       bf16 [M, N]  (written; must not overlap the inputs)
  *   y[m][n] = sum_k x[m][k] * w_hat[n][k]
  *
- * M = 3 .. 16 with 2-, 4- or 8-bit codes (K a multiple of 1024/bits,
- * K/group_size a multiple of 8) runs on the tensor cores: each w_hat is
- * rounded once to fp16 and each x row is scaled by a power of two into fp16
- * range, with fp32 accumulation; scales and biases should lie in fp16's
- * normal range (magnitude 2^-14 .. 65504) there.  The first such call on a
- * device allocates the path's scratch (2.4 MB plus 4 bytes per 128 rows);
- * qmv_noalloc does the same without allocating.
+ * With 2-, 4- or 8-bit codes, K a multiple of 1024/bits and K/group_size a
+ * multiple of 8, several activation rows run on the tensor cores:
+ *   M = 3 .. 16: each w_hat is rounded once to fp16 and each x row is scaled
+ *     by a power of two into fp16 range, with fp32 accumulation; scales and
+ *     biases should lie in fp16's normal range (magnitude 2^-14 .. 65504);
+ *   M >= 17 (the pages' qmm_t, "quantized.h": qmm_t_impl / affine_qmm_t):
+ *     bf16 operands, w_hat = bf16(scale * q + bias) rounded once (the value
+ *     dequantize writes), x as given, fp32 accumulation; blocks of 32, 64 or
+ *     128 activation rows.
+ * The first such call on a device allocates the paths' scratch (split-tile
+ * partial sums: 2 x SMs x rows-per-block x 128 floats, at most 19.4 MB on a
+ * 148-SM GPU, plus 4 bytes per tile); qmv_noalloc does the same without
+ * allocating.
  */
 int qmv(const void *x, const uint32_t *w, const void *scales,
         const void *biases, void *y, int M, int N, int K, int bits,
@@ -94,9 +100,11 @@ int qmv(const void *x, const uint32_t *w, const void *scales,
  * device memory allocated by the library.  qmv's tensor-core path (several
  * activation rows, 2/4/8-bit codes) adds up 128-row tiles that are split
  * between CTAs through scratch memory the library allocates on first use;
- * qmv_noalloc takes that scratch from a fixed array in the library's device
- * image instead (its address from cudaGetSymbolAddress, per device).
- * Results are identical to qmv's for the same inputs.
+ * for M = 3 .. 16 qmv_noalloc takes that scratch from a fixed array in the
+ * library's device image instead (its address from cudaGetSymbolAddress, per
+ * device), with results identical to qmv's; for M >= 17 it gives every CTA
+ * whole tiles and needs no scratch at all (the same result within the
+ * accuracy bound; the fp32 sums run in another order than qmv's).
  *   returns QMV_ERR_UNSUPPORTED when the call would need more than the array
  *   holds: more than 256 SMs, or more than 65536 row tiles (N > 8388608).
  * Calls on one device that use the array are expected in stream order.

@@ -219,3 +219,22 @@ def test_qvm_workload_arrays_have_the_launch_shapes():
     assert l.x.shape == (l.M, l.K)
     assert l.w.shape == (l.K, l.N * l.bits // 32) and l.s.shape == (l.K, l.N // l.gs)
     assert l.nbytes == _arrays_bytes(l.w, l.s, l.b, l.x) + 2 * l.M * l.N
+
+
+def test_roofline_takes_the_longer_of_memory_and_tensor_time():
+    # a launch whose FLOPs at the tensor peak take longer than its bytes at
+    # the HBM peak is tensor bound; otherwise memory bound
+    L = bench.Launch("t", "qmv", nbytes=1_000_000, flops=2 * 128 * 28672 * 8192)
+    r = bench._roofline(L, 0.1, 6537.0, "measured", 1627.7, "measured", "b", None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - L.flops / 1e-4 / 1e12) < 0.1
+    L2 = bench.Launch("m", "qmv", nbytes=147_000_000, flops=2 * 32 * 28672 * 8192)
+    r2 = bench._roofline(L2, 0.05, 6537.0, "measured", 1627.7, "measured", "b", None)
+    assert r2["bound"] == "hbm" and r2["unit"] == "GB/s"
+
+
+def test_prefill_launches_carry_their_flops():
+    launches, cfg = bench.workload("prefill")
+    for l in launches:
+        assert l.flops == 2 * l.M * l.N * l.K
+        assert l.nbytes == _arrays_bytes(l.w, l.s, l.b, l.x) + 2 * l.M * l.N

@@ -1,13 +1,22 @@
-"""qmv_noalloc: the same results as qmv, with the tensor-core path's
+"""qmv_noalloc: the same results as qmv, with the few-row tensor-core path's
 split-tile scratch taken from the library's fixed device array instead of an
-allocation.  Collected last, so the allocating entry point has run first."""
+allocation, and the many-row path on whole tiles (no scratch at all).
+Collected last, so the allocating entry point has run first."""
 import numpy as np
 import pytest
 import torch
 
 import affine_group_quantized_b200 as agq
 from affine_group_quantized_b200 import synth
-from tests._parity import dev_bf16, dev_u32, empty_bf16, host_bits
+import oracle
+from tests._parity import check, dev_bf16, dev_u32, empty_bf16, host_bits, sample_rows
+
+
+def _run(fn, x, w, s, b, M, N, K, bits, gs):
+    Y = empty_bf16(M, N)
+    fn(dev_bf16(x), dev_u32(w), dev_bf16(s), dev_bf16(b), Y, M, N, K, bits, gs)
+    torch.cuda.synchronize()
+    return host_bits(Y)
 
 
 def test_noalloc_is_exported_and_bound():
@@ -55,3 +64,22 @@ def test_noalloc_matches_qmv_twice_in_a_row(M, N, K, bits, gs):
         outs.append(host_bits(Y))
     for o in outs[1:]:
         assert np.array_equal(outs[0], o)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M, N, K, bits, gs", [
+    (48, 150 * 128 - 20, 1024, 4, 32),   # more tiles than SMs
+    (130, 300, 2048, 8, 64),             # two column blocks
+    (20, 700, 2048, 2, 128),
+])
+def test_noalloc_many_rows_whole_tiles(M, N, K, bits, gs):
+    # without scratch every CTA takes whole tiles; the sums then run in
+    # another order than with split tiles, so compare with the oracle, and
+    # with itself
+    x, w, s, b = synth.qmv_inputs(M, N, K, bits, gs, seed=8600 + M + bits)
+    y1 = _run(agq.qmv_noalloc, x, w, s, b, M, N, K, bits, gs)
+    y2 = _run(agq.qmv_noalloc, x, w, s, b, M, N, K, bits, gs)
+    assert np.array_equal(y1, y2)
+    rows = sample_rows(N, 400, seed=M) if N > 400 else None
+    y_ref, a_ref = oracle.qmv(x, w, s, b, M, N, K, bits, gs, rows=rows, nthreads=8)
+    check(y1 if rows is None else y1[:, rows], y_ref, a_ref, f"qmm noalloc M={M}")
