@@ -47,11 +47,18 @@ namespace qmvk {
 
 template <int MC>
 struct QmmShape {
-  // independent accumulators per tile (small MMAs go round-robin)
-  static constexpr int kNacc = MC >= 64 ? 1 : 64 / MC;
-  static constexpr int kDCols = 2 * kNacc * MC;  // double-buffered
+  // MMA-issuing warps: a thread issues an MMA about every 25 ns whatever its
+  // size, while the tensor core takes one of N <= 64 in about 10-18 ns, so
+  // narrow blocks spread their chunks over two issuers (chunk j of a segment
+  // goes to issuer j % 2), each with its own accumulator; the epilogue adds
+  // them in issuer order
+  static constexpr int kIssuers = MC >= 128 ? 1 : 2;
+  static constexpr int kNacc = 1;                         // accumulators per issuer
+  static constexpr int kDCols = 2 * kIssuers * MC;        // double-buffered
   static constexpr int kAbufs = (512 - kDCols) / 64 < 7 ? (512 - kDCols) / 64 : 7;
   static constexpr uint32_t kDCol = kAbufs * 64;  // first accumulator column
+  // accumulator of issuer i in buffer db
+  static constexpr uint32_t dcol(int db, int i) { return kDCol + (db * kIssuers + i) * MC; }
   static constexpr uint32_t kXBytes = MC * 256;   // one x chunk: MC rows x 128 k bf16
   // fp32 D, bf16 A and B, both K-major, N = MC, M = 128
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -89,7 +96,8 @@ template <int BITS>
 __host__ __device__ constexpr int qmm_part_codes() { return QmmStage<BITS>::SC / kQmmParts; }
 template <int BITS>
 __host__ __device__ constexpr int qmm_warps_per_chunk() { return 4 * (kMmaKC / qmm_part_codes<BITS>()); }
-constexpr int kQmmThreads = (4 * kQmmParts + 2) * 32;
+template <int MC>
+__host__ __device__ constexpr int qmm_threads() { return (4 * kQmmParts + 1 + QmmShape<MC>::kIssuers) * 32; }
 
 struct QmmSmem {
   // wfull, wempty [kMmaMaxStages]; xfull, xempty [kQmmMaxX];
@@ -148,6 +156,50 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t tmem_d, uint32_t tmem_a, u
       "}\n" ::"r"(tmem_d),
       "r"(tmem_a), "l"(db), "r"(QmmShape<MC>::kIdesc), "r"(accumulate), "r"(0u), "r"(0u),
       "r"(0u), "r"(0u)
+      : "memory");
+}
+
+// The eight K = 16 MMAs of one 128-k chunk, all accumulating, from one asm
+// block with their operands formed inside it: A at tensor-memory columns
+// a0 + 8j; B's descriptor start field (16-byte units; shared addresses stay
+// below 2^18, so the low word never carries) at box j / 4 of the chunk
+// (MC * 128 bytes apart) and 32 bytes (16 k) per j inside the swizzled row;
+// D round-robin over the accumulators (MC columns apart).  Few instructions
+// per MMA matter: the issuing thread shares its scheduler with dequant warps.
+template <int MC>
+__device__ __forceinline__ void umma_chunk_acc(uint32_t d0, uint32_t a0, uint64_t b0) {
+  constexpr int NA = QmmShape<MC>::kNacc;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      ".reg .b32 bl, bh, t;\n"
+      ".reg .b32 a1, a2, a3, a4, a5, a6, a7;\n"
+      ".reg .b32 d1, d2, d3;\n"
+      ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n"
+      "setp.ne.b32 p, 1, 0;\n"
+      "mov.b64 {bl, bh}, %2;\n"
+      "add.u32 a1, %1, 8;\n add.u32 a2, %1, 16;\n add.u32 a3, %1, 24;\n add.u32 a4, %1, 32;\n"
+      "add.u32 a5, %1, 40;\n add.u32 a6, %1, 48;\n add.u32 a7, %1, 56;\n"
+      "add.u32 t, bl, 2;\n mov.b64 b1, {t, bh};\n"
+      "add.u32 t, bl, 4;\n mov.b64 b2, {t, bh};\n"
+      "add.u32 t, bl, 6;\n mov.b64 b3, {t, bh};\n"
+      "add.u32 t, bl, %4;\n mov.b64 b4, {t, bh};\n"
+      "add.u32 t, bl, %5;\n mov.b64 b5, {t, bh};\n"
+      "add.u32 t, bl, %6;\n mov.b64 b6, {t, bh};\n"
+      "add.u32 t, bl, %7;\n mov.b64 b7, {t, bh};\n"
+      "add.u32 d1, %0, %8;\n add.u32 d2, %0, %9;\n add.u32 d3, %0, %10;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b1, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d2], [a2], b2, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d3], [a3], b3, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d1], [a5], b5, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d2], [a6], b6, %3, p;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [d3], [a7], b7, %3, p;\n"
+      "}\n" ::"r"(d0),
+      "r"(a0), "l"(b0), "r"(QmmShape<MC>::kIdesc), "n"(MC * 8), "n"(MC * 8 + 2),
+      "n"(MC * 8 + 4), "n"(MC * 8 + 6), "n"((1 % NA) * MC), "n"((2 % NA) * MC),
+      "n"((3 % NA) * MC)
       : "memory");
 }
 
@@ -216,7 +268,7 @@ __device__ __forceinline__ void unpack_word_bf16(uint32_t w, uint32_t s2, uint32
 }
 
 template <int BITS, int GS, int MC>
-__global__ void __launch_bounds__(kQmmThreads, 1)
+__global__ void __launch_bounds__(qmm_threads<MC>(), 1)
     qmm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x,
                const QmmParams p) {
@@ -258,7 +310,7 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
       mbar_init(&abempty[lane], 1);  // tcgen05.commit
     }
     if (lane < 2) {
-      mbar_init(&dfull[lane], 1);    // tcgen05.commit
+      mbar_init(&dfull[lane], SH::kIssuers);  // a tcgen05.commit per issuer
       mbar_init(&dempty[lane], nw);  // every dequant warp
     }
     fence_mbar_init();
@@ -369,10 +421,11 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
       if (dead && p.err) atomicOr(p.err, 2);
     }
     __syncwarp();
-  } else if (warp == nw + 1) {
-    // ---------------- MMA warp ----------------
+  } else if (warp > nw) {
+    // ---------------- MMA warps ----------------
+    const int issuer = warp - nw - 1;
     RingPos ap, xp;
-    int sidx = 0;
+    int sidx = 0, jj = 0;  // segments done; chunk index inside the segment
     bool dead = false;
     const uint64_t xdesc0 = sw128_desc(xring);
     int c = static_cast<int>(v0 % p.nstage);
@@ -382,14 +435,20 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
     for (long long v = v0; v < v1; ++v) {
       if (seg_start) {
         db = sidx & 1;
+        jj = 0;
         const uint32_t dph = static_cast<uint32_t>((sidx >> 1) & 1);
         if (sidx >= 2 && !dead && !mbar_wait_sleep(&dempty[db], dph ^ 1u)) dead = true;
         tc_fence_after();
-        tmem_d = tmem_base + SH::kDCol + db * (SH::kNacc * MC);
+        tmem_d = tmem_base + SH::dcol(db, issuer);
       }
       const bool seg_end = (c == p.nstage - 1) || (v == v1 - 1);
 #pragma unroll 1
-      for (int h = 0; h < CPS; ++h) {
+      for (int h = 0; h < CPS; ++h, ++jj) {
+        if (jj % SH::kIssuers != issuer) {  // another issuer's chunk
+          ap.next(NAB);
+          xp.next(nxs);
+          continue;
+        }
         if (!dead && !mbar_wait_sleep(&abfull[ap.idx], ap.phase)) dead = true;
         if (!dead && !mbar_wait_sleep(&xfull[xp.idx], xp.phase)) dead = true;
         tc_fence_after();
@@ -399,22 +458,30 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
           // (shared addresses stay below 2^18): box j / 4 of the chunk,
           // 32 bytes (16 k) per MMA inside the 128-byte swizzled row
           const uint64_t d0 = xdesc0 + static_cast<uint64_t>((xp.idx * SH::kXBytes) >> 4);
-          const bool first = seg_start && h == 0;
+          if (jj < SH::kIssuers) {
+            // this issuer's first chunk of the segment: its first MMA into
+            // each accumulator overwrites it
 #pragma unroll
-          for (int j = 0; j < kMmaKC / 16; ++j) {
-            const uint64_t dj =
-                d0 + static_cast<uint64_t>(((j >> 2) * MC * 128 + (j & 3) * 32) >> 4);
-            umma_bf16_ta<MC>(tmem_d + (j % SH::kNacc) * MC, a0 + j * 8, dj,
-                             (first && j < SH::kNacc) ? 0u : 1u);
+            for (int j = 0; j < kMmaKC / 16; ++j) {
+              const uint64_t dj =
+                  d0 + static_cast<uint64_t>(((j >> 2) * MC * 128 + (j & 3) * 32) >> 4);
+              umma_bf16_ta<MC>(tmem_d + (j % SH::kNacc) * MC, a0 + j * 8, dj,
+                               j < SH::kNacc ? 0u : 1u);
+            }
+          } else {
+            umma_chunk_acc<MC>(tmem_d, a0, d0);
           }
           mma_commit(&abempty[ap.idx]);
           mma_commit(&xempty[xp.idx]);
-          if (seg_end && h == CPS - 1) mma_commit(&dfull[db]);
         }
         __syncwarp();
         ap.next(NAB);
         xp.next(nxs);
       }
+      // every issuer signals the segment's end, with or without chunks in
+      // it (the commit covers all of this thread's earlier MMAs)
+      if (seg_end && lane == 0) mma_commit(&dfull[db]);
+      __syncwarp();
       if (seg_end) ++sidx;
       seg_start = seg_end;
       if (++c == p.nstage) c = 0;
@@ -508,6 +575,7 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
       // the next stage of this CTA's walk
       const int tc = t;
       const bool seg_end = (c == p.nstage - 1) || (v == v1 - 1);
+      const int seg_chunks = (c - cseg0 + 1) * CPS;  // when seg_end: the segment's chunks
       const bool whole_tile = seg_end && cseg0 == 0 && c == p.nstage - 1;
       ++v;
       if (++c == p.nstage) {
@@ -532,7 +600,10 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
         const uint32_t dph = static_cast<uint32_t>((sidx >> 1) & 1);
         if (!dead && !mbar_wait(&dfull[db], dph)) dead = true;
         tc_fence_after();
-        const uint32_t dcol = tmem_base + lane_q + SH::kDCol + db * (SH::kNacc * MC);
+        const uint32_t dcol = tmem_base + lane_q + SH::dcol(db, 0);
+        // issuers that had chunks in the segment (the others' accumulators
+        // hold an older segment)
+        const int used = seg_chunks < SH::kIssuers ? seg_chunks : SH::kIssuers;
         const int rt = 32 * (warp % 4) + lane;  // row in the tile
         const int nt = tc / p.nmb, mb = tc - nt * p.nmb;
         const int row = nt * kMmaRows + rt;
@@ -540,11 +611,13 @@ __global__ void __launch_bounds__(kQmmThreads, 1)
         auto read_piece = [&](int pc, float (&d)[16]) {
           tmem_ld16(dcol + 16 * pc, d);
 #pragma unroll
-          for (int a = 1; a < SH::kNacc; ++a) {
-            float e[16];
-            tmem_ld16(dcol + a * MC + 16 * pc, e);
+          for (int a = 1; a < SH::kIssuers; ++a) {
+            if (a < used) {  // warp-uniform
+              float e[16];
+              tmem_ld16(dcol + a * MC + 16 * pc, e);
 #pragma unroll
-            for (int m = 0; m < 16; ++m) d[m] += e[m];
+              for (int m = 0; m < 16; ++m) d[m] += e[m];
+            }
           }
         };
         if (whole_tile) {
@@ -733,7 +806,7 @@ int launch_t(const QmmArgs &a, char *msg, size_t n) {
   const long long grid = tiles * p.nstage < a.sms ? tiles * p.nstage : a.sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.part ? grid : (tiles < a.sms ? tiles : a.sms)));
-  cfg.blockDim = dim3(qmvk::kQmmThreads);
+  cfg.blockDim = dim3(qmvk::qmm_threads<MC>());
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = a.stream;
   cudaLaunchAttribute attr[1];
