@@ -214,8 +214,11 @@ int qmv_silu_gate_resid(const void *gate, const void *up, const void *x_resid,
  *                row unwritten; valid pairs are still computed.  A bounded
  *                wait that gave up ORs 2 (see Conventions).  The caller
  *                zeroes *d_status before the call.
- * The kernel reads every expert that some pair uses once per call, whether or
- * not the indices are sorted.  num_pairs may be 0 (nothing is enqueued).
+ * The kernel groups the pairs by expert itself (so sorting is only a hint)
+ * and streams a touched expert's rows once per two of its pairs: an expert
+ * with c pairs is read ceil(c / 2) times, its reads next to each other in
+ * the launch so that the later ones mostly come from L2; untouched experts
+ * are not read.  num_pairs may be 0 (nothing is enqueued).
  */
 int gather_qmv(const void *x, const uint32_t *w, const void *scales,
                const void *biases, const uint32_t *lhs_indices,
