@@ -844,6 +844,74 @@ int launch_qvm_t(const qmvk::QvmParams &p, cudaStream_t stream) {
   return ok();
 }
 
+// The staged qvm: rows streamed by the tensor-copy engine.  Needs the code
+// and scale rows to be multiples of 16 bytes (N * bits % 128 == 0 and
+// (N / gs) % 8 == 0); other shapes take qvm_kernel.
+// Dynamic shared memory of the staged qvm: the CTA's activations (fp32),
+// 128 bytes of alignment slack, the stages.
+int qvm_tma_smem(int K, int bits, uint32_t *ring_off, uint32_t *stage_bytes) {
+  const int xrows = (K + qmvk::kQvmCluster - 1) / qmvk::kQvmCluster + 1;
+  *ring_off = static_cast<uint32_t>((4LL * xrows + 127) / 128 * 128);
+  *stage_bytes = static_cast<uint32_t>(qmvk::kQvtRows * 32 * bits + 2 * qmvk::kQvtRows * 16);
+  return static_cast<int>(*ring_off) + 128 + qmvk::kQvtStages * static_cast<int>(*stage_bytes);
+}
+// the staged kernel's static shared memory (partials, barriers), with room
+constexpr int kQvtStaticSmem = 20 * 1024;
+
+template <int BITS>
+int launch_qvm_tma_t(const qmvk::QvmParams &q, DeviceInfo *dev, cudaStream_t stream) {
+  constexpr int WB = 32 * BITS;
+  qmvk::QvtParams p;
+  std::memset(&p, 0, sizeof p);
+  p.y = q.y;
+  p.x = q.x;
+  p.err = dev->status;
+  p.M = q.M;
+  p.K = q.K;
+  p.N = q.N;
+  p.gs_shift = q.gs_shift;
+  p.x_off = 0;
+  const int smem = qvm_tma_smem(q.K, BITS, &p.ring_off, &p.stage_bytes);
+  CUtensorMap tw, ts, tb;
+  int rc;
+  if ((rc = encode_2d(&tw, q.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, q.row_bytes, q.K, q.row_bytes, WB,
+                      qmvk::kQvtRows, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B)))
+    return rc;
+  if ((rc = encode_2d(&ts, q.s, CU_TENSOR_MAP_DATA_TYPE_UINT16, q.G, q.K, 2ull * q.G, 8,
+                      qmvk::kQvtRows, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)))
+    return rc;
+  if ((rc = encode_2d(&tb, q.b, CU_TENSOR_MAP_DATA_TYPE_UINT16, q.G, q.K, 2ull * q.G, 8,
+                      qmvk::kQvtRows, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)))
+    return rc;
+  auto kern = qmvk::qvm_tma_kernel<BITS>;
+  int d = 0;
+  cudaGetDevice(&d);
+  static int granted[kMaxDevices] = {};
+  if (smem > 48 * 1024 && smem > granted[d]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+      return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    granted[d] = smem;
+  }
+  const int nblk = (q.N + qmvk::kQvmCols - 1) / qmvk::kQvmCols;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nblk, qmvk::kQvmCluster, q.M);
+  cfg.blockDim = dim3((qmvk::kQvtWarps + 1) * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tw, ts, tb, p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();  // clear it
+    return fail(QMV_ERR_CUDA, "qvm launch: %s", cudaGetErrorString(le));
+  }
+  return ok();
+}
+
 // ---------------------------------------------------------------------------
 // Trellis mode (qmv_trellis.cuh)
 // ---------------------------------------------------------------------------
@@ -948,6 +1016,19 @@ int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases
   p.gs_shift = group_size == 32 ? 5 : group_size == 64 ? 6 : 7;
   p.row_bytes = static_cast<uint32_t>(static_cast<long long>(N) * bits / 8);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t ro, sbytes;
+  if ((static_cast<long long>(N) * bits) % 128 == 0 && p.G % 8 == 0 &&
+      qvm_tma_smem(K, bits, &ro, &sbytes) <= dev->smem_optin - kQvtStaticSmem) {
+    switch (bits) {
+      case 2: return launch_qvm_tma_t<2>(p, dev, st);
+      case 3: return launch_qvm_tma_t<3>(p, dev, st);
+      case 4: return launch_qvm_tma_t<4>(p, dev, st);
+      case 5: return launch_qvm_tma_t<5>(p, dev, st);
+      case 6: return launch_qvm_tma_t<6>(p, dev, st);
+      case 8: return launch_qvm_tma_t<8>(p, dev, st);
+      default: break;
+    }
+  }
   switch (bits) {
     case 2: return launch_qvm_t<2>(p, st);
     case 3: return launch_qvm_t<3>(p, st);

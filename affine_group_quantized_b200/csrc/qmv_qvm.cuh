@@ -23,6 +23,7 @@
 #include <cooperative_groups.h>
 
 #include "qmv_device.cuh"
+#include "qmv_mma.cuh"
 
 namespace qmvk {
 
@@ -170,6 +171,159 @@ __global__ void __cluster_dims__(1, kQvmCluster, 1) __launch_bounds__(kQvmWarps 
     }
   }
   cluster.sync();  // the other CTAs keep their shared memory until it was read
+}
+
+// ---------------------------------------------------------------------------
+// The staged form (row strides a multiple of 16 bytes): the same lanes,
+// column blocks and cluster row split, with the rows streamed into shared
+// memory by the tensor-copy engine.  A CTA's rows are one contiguous range;
+// per stage one thread copies kQvtRows rows of the block's 32 * BITS bytes
+// (2-D box, rows past K arrive as zeros) and the rows' 16-byte scale and
+// bias windows (8 groups from the block's first group rounded down to a
+// multiple of 8); sixteen consumer warps take the stage's rows in turn.
+// Long copies of many rows keep enough bytes in flight to stream at HBM
+// speed, where per-lane loads of a few bytes per row did not.
+// ---------------------------------------------------------------------------
+constexpr int kQvtRows = 64;    // rows per stage
+constexpr int kQvtWarps = 16;   // consumer warps
+constexpr int kQvtStages = 8;   // stages in the ring
+
+struct QvtParams {
+  uint16_t *y;            // bf16 [M][N]
+  const uint16_t *x;      // bf16 [M][K]
+  int *err;               // OR 2 when a bounded wait gave up
+  int M, K, N;
+  int gs_shift;           // log2(group size)
+  uint32_t stage_bytes;   // W rows, then the scale and bias windows
+  uint32_t x_off;         // smem offset of the CTA's activations (fp32)
+  uint32_t ring_off;      // smem offset of the stages (rounded up to 128 in the kernel)
+};
+
+template <int BITS>
+__global__ void __cluster_dims__(1, kQvmCluster, 1) __launch_bounds__((kQvtWarps + 1) * 32, 1)
+    qvm_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                   const __grid_constant__ CUtensorMap tm_b, const QvtParams p) {
+  namespace cg = cooperative_groups;
+  constexpr int WB = 32 * BITS;                     // bytes of a row in the block
+  constexpr uint32_t kSOff = kQvtRows * WB;         // scale windows [rows][16 B]
+  constexpr uint32_t kBOff = kSOff + kQvtRows * 16; // bias windows
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ float red[kQvtWarps][kQvmCols];
+  __shared__ float part[kQvmCols];
+  __shared__ uint64_t bars[2 * kQvtStages];
+  uint64_t *full = bars, *empty = bars + kQvtStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = blockIdx.x, rank = blockIdx.y, m = blockIdx.z;
+  const int c = nb * 32 + lane;               // this lane's chunk of 8 columns
+  const bool live = 8 * c < p.N;
+  const int k0 = static_cast<int>(static_cast<long long>(p.K) * rank / kQvmCluster);
+  const int k1 = static_cast<int>(static_cast<long long>(p.K) * (rank + 1) / kQvmCluster);
+  const int nstg = (k1 - k0 + kQvtRows - 1) / kQvtRows;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t ring = (sbase + p.ring_off + 127u) & ~127u;  // 128 bytes of slack
+  float *xs = reinterpret_cast<float *>(smem + p.x_off);
+  const int gwin = ((nb * kQvmCols) >> p.gs_shift) & ~7;  // first group of the windows
+  grid_launch_dependents();
+  if (warp == kQvtWarps) {
+    if (lane < kQvtStages) {
+      mbar_init(&full[lane], 1);
+      mbar_init(&empty[lane], kQvtWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dependency_wait();
+
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  float bacc = 0.f;
+  bool dead = false;
+  if (warp == kQvtWarps) {
+    // ---- producer (one thread) ----
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      for (int j = 0; j < nstg; ++j) {
+        const int slot = j % kQvtStages;
+        if (j >= kQvtStages && !dead &&
+            !mbar_wait_sleep(&empty[slot], static_cast<uint32_t>(((j / kQvtStages) - 1) & 1)))
+          dead = true;
+        const uint32_t dst = ring + slot * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[slot], p.stage_bytes);
+        const int kr = k0 + j * kQvtRows;
+        tma_load_2d(dst, &tm_w, nb * WB, kr, &full[slot], pol);
+        tma_load_2d(dst + kSOff, &tm_s, gwin, kr, &full[slot], pol);
+        tma_load_2d(dst + kBOff, &tm_b, gwin, kr, &full[slot], pol);
+      }
+      // every copy lands before the CTA exits
+      for (int j = nstg - kQvtStages < 0 ? 0 : nstg - kQvtStages; j < nstg; ++j)
+        if (!dead && !mbar_wait_sleep(&full[j % kQvtStages],
+                                      static_cast<uint32_t>((j / kQvtStages) & 1)))
+          dead = true;
+      if (dead && p.err) atomicOr(p.err, 2);
+    }
+    __syncwarp();
+  } else {
+    // ---- consumers: the CTA's activations, then the stages ----
+    const uint16_t *xr = p.x + static_cast<size_t>(m) * p.K;
+    for (int k = k0 + static_cast<int>(threadIdx.x); k < k1; k += kQvtWarps * 32)
+      xs[k - k0] = bf16_to_f32(xr[k]);
+    named_sync(1, kQvtWarps * 32);
+    const int gl = ((8 * c) >> p.gs_shift) - gwin;  // the chunk's group in the window
+    const uint32_t cb = static_cast<uint32_t>(lane) * BITS;  // the chunk's bytes in a row
+    for (int j = 0; j < nstg; ++j) {
+      const int slot = j % kQvtStages;
+      if (!dead && !mbar_wait(&full[slot], static_cast<uint32_t>((j / kQvtStages) & 1)))
+        dead = true;
+      const uint32_t stg = ring + slot * p.stage_bytes;
+      const int kr = k0 + j * kQvtRows;
+      if (live) {
+#pragma unroll 4
+        for (int r = warp; r < kQvtRows; r += kQvtWarps) {
+          const int k = kr + r;
+          if (k >= k1) break;
+          const uint32_t ra = stg + static_cast<uint32_t>(r) * WB;
+          // the chunk's BITS bytes as the aligned words that hold them
+          const uint32_t a0 = ra + (cb & ~3u);
+          uint64_t v = lds32(a0);
+          if ((cb & 3u) + BITS > 4) v |= static_cast<uint64_t>(lds32(a0 + 4)) << 32;
+          v >>= 8 * (cb & 3u);
+          const float xk = xs[k - k0];
+          const float sk = bf16_to_f32(static_cast<uint16_t>(lds16(stg + kSOff + r * 16 + 2 * gl)));
+          const float bk = bf16_to_f32(static_cast<uint16_t>(lds16(stg + kBOff + r * 16 + 2 * gl)));
+          bacc = fmaf(xk, bk, bacc);
+          qvm_row<BITS>(v, xk * sk, acc);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    if (dead && p.err && lane == 0) atomicOr(p.err, 2);
+  }
+  // columns of this warp's partials, then the CTA's sum in warp order
+  if (warp < kQvtWarps) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      red[warp][8 * lane + 2 * j] = acc[j].x + bacc;
+      red[warp][8 * lane + 2 * j + 1] = acc[j].y + bacc;
+    }
+  }
+  __syncthreads();
+  for (int col = threadIdx.x; col < kQvmCols; col += blockDim.x) {
+    float sum = 0.f;
+    for (int w = 0; w < kQvtWarps; ++w) sum += red[w][col];
+    part[col] = sum;
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  if (rank == 0) {
+    for (int col = threadIdx.x; col < kQvmCols; col += blockDim.x) {
+      const int n = nb * kQvmCols + col;
+      float sum = 0.f;
+      for (int r = 0; r < kQvmCluster; ++r) sum += cluster.map_shared_rank(part, r)[col];
+      if (n < p.N) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16(sum);
+    }
+  }
+  cluster.sync();
 }
 
 }  // namespace qmvk

@@ -72,3 +72,17 @@ def test_qvm_repeatable():
     x, w, s, b = _inputs(M, K, N, bits, gs, seed=9)
     ys = [_qvm(x, w, s, b, M, K, N, bits, gs) for _ in range(3)]
     assert all(np.array_equal(ys[0], y) for y in ys[1:])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_qvm_staged_shapes(bits, gs):
+    # shapes whose code and scale rows are whole 16-byte units (the staged
+    # kernel): rows that split unevenly between the cluster's CTAs and the
+    # 64-row stages, CTAs with a single short stage, CTAs with no rows
+    for (M, K, N) in [(2, 1000, 1024), (1, 70, 2048), (1, 7, 1024), (3, 4099, 3072)]:
+        assert (N * bits) % 128 == 0 and (N // gs) % 8 == 0
+        x, w, s, b = _inputs(M, K, N, bits, gs, seed=bits * 57 + gs + K)
+        y = _qvm(x, w, s, b, M, K, N, bits, gs)
+        y_ref, a_ref = oracle.qvm(x, w, s, b, M, K, N, bits, gs)
+        check(y, y_ref, a_ref, f"qvm staged bits={bits} gs={gs} M={M} K={K} N={N}")
