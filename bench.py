@@ -375,7 +375,8 @@ class ClockSampler:
 # recorded DRAM traffic is valid while these are unchanged.  (The producer
 # side of the format, qmv_quant.cu, has kernels of its own.)
 GEMV_SOURCES = ("qmv_api.cu", "qmv_decode.cuh", "qmv_device.cuh", "qmv_mma.cuh",
-                "qmv_stream.cuh")
+                "qmv_qmm.cu", "qmv_qmm.h", "qmv_quant.cu", "qmv_qvm.cuh", "qmv_stream.cuh",
+                "qmv_trellis.cuh")
 
 
 def source_hash():

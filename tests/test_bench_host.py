@@ -158,7 +158,7 @@ def test_recorded_traffic_only_for_the_captured_source(monkeypatch, tmp_path):
                                      "dram_bytes_per_launch": 33067008}}}))
     assert bench.recorded_traffic("qmv_b4", "decode_sweep") == 33067008
     assert bench.recorded_traffic("qmv_b8", "decode_sweep") is None
-    (csrc / "qmv_quant.cu").write_text("other kernels\n")   # not a GEMV source
+    (csrc / "notes.txt").write_text("not a kernel source\n")
     assert bench.source_hash() == h
     assert bench.recorded_traffic("qmv_b4", "decode_sweep") == 33067008
     (csrc / "qmv_stream.cuh").write_text("kernel v2\n")     # source changed since
