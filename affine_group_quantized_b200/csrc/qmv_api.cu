@@ -928,7 +928,7 @@ int launch_trellis_t(const qmvk::TrellisParams &p, int sms, cudaStream_t stream)
       return fail(QMV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     granted[dev] = smem;
   }
-  const int rows_per_cta = qmvk::kTrellisWarps;
+  const int rows_per_cta = qmvk::kTrellisWarps * qmvk::trellis_rows_per_warp<BITS>();
   long long grid = (p.N + rows_per_cta - 1) / rows_per_cta;
   if (grid > 16LL * sms) grid = 16LL * sms;
   cudaLaunchConfig_t cfg = {};

@@ -13,9 +13,11 @@
 // as binary16 numbers (one binary16 rounding).  There are no groups and no
 // biases: one scale serves the matrix.
 //
-// A warp takes a row at a time; a lane takes chunks of 8 words (one 16-byte
-// load) plus the word after them, so each word's successor is at hand.  The
-// activation row sits in shared memory as fp32.  Each value is a few integer
+// A warp takes four or eight rows at a time; a lane takes chunks of 8 words
+// (one 16-byte load per row) plus the word after them, so each word's
+// successor is at hand.  The activation row sits in shared memory as fp32;
+// a word's activations are read once (16-byte loads) for all the warp's
+// rows.  Each value is a few integer
 // and one binary16 operation away from its state; products and sums are
 // fp32, reduced over the warp with shuffles, scaled and rounded once to
 // bf16.
@@ -65,11 +67,16 @@ __device__ __forceinline__ float trellis_word(uint32_t w0, uint32_t w1, const fl
   return acc;
 }
 
+// Rows a warp works on at once: they share every activation load.
+template <int BITS>
+__host__ __device__ constexpr int trellis_rows_per_warp() { return BITS == 4 ? 8 : 4; }
+
 template <int BITS>
 __global__ void __launch_bounds__(kTrellisWarps * 32)
     qmv_trellis_kernel(const TrellisParams p) {
   extern __shared__ __align__(16) float xs[];  // the activation row, fp32 [K]
   constexpr int C = 16 / BITS;
+  constexpr int RW = trellis_rows_per_warp<BITS>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.y;
   grid_launch_dependents();
@@ -79,22 +86,59 @@ __global__ void __launch_bounds__(kTrellisWarps * 32)
   __syncthreads();
   const float scale = bf16_to_f32(p.scales[0]);
   const int nchunks = p.W / 8;  // 8-word chunks per row
-  for (int n = blockIdx.x * kTrellisWarps + warp; n < p.N; n += gridDim.x * kTrellisWarps) {
-    const uint16_t *row = p.w + static_cast<size_t>(n) * p.W;
-    float acc = 0.f;
-    for (int ch = lane; ch < nchunks; ch += 32) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row) + ch);
-      const int after = (8 * ch + 8) % p.W;  // the word after the chunk
-      const uint32_t next = __ldg(row + after);
-      const uint32_t u[9] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16, v.z & 0xFFFFu,
-                             v.z >> 16,     v.w & 0xFFFFu, v.w >> 16, next};
+  const int stride = gridDim.x * kTrellisWarps * RW;
+  for (int n0 = (blockIdx.x * kTrellisWarps + warp) * RW; n0 < p.N; n0 += stride) {
+    // RW rows (past N: row n0 again, its sums dropped)
+    const uint16_t *row[RW];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc += trellis_word<BITS>(u[i], u[i + 1], xs + (8 * ch + i) * C);
+    for (int r = 0; r < RW; ++r)
+      row[r] = p.w + static_cast<size_t>(n0 + r < p.N ? n0 + r : n0) * p.W;
+    float acc[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r) acc[r] = 0.f;
+    for (int ch = lane; ch < nchunks; ch += 32) {
+      const int after = (8 * ch + 8) % p.W;  // the word after the chunk
+      uint32_t u[RW][9];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row[r]) + ch);
+        u[r][0] = v.x & 0xFFFFu;
+        u[r][1] = v.x >> 16;
+        u[r][2] = v.y & 0xFFFFu;
+        u[r][3] = v.y >> 16;
+        u[r][4] = v.z & 0xFFFFu;
+        u[r][5] = v.z >> 16;
+        u[r][6] = v.w & 0xFFFFu;
+        u[r][7] = v.w >> 16;
+        u[r][8] = __ldg(row[r] + after);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // the word's C activations, read once for the RW rows
+        float xv[C];
+        const float4 *xp = reinterpret_cast<const float4 *>(xs + (8 * ch + i) * C);
+#pragma unroll
+        for (int q = 0; q < C / 4; ++q) {
+          const float4 f = xp[q];
+          xv[4 * q] = f.x;
+          xv[4 * q + 1] = f.y;
+          xv[4 * q + 2] = f.z;
+          xv[4 * q + 3] = f.w;
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r) acc[r] += trellis_word<BITS>(u[r][i], u[r][i + 1], xv);
+      }
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16(scale * acc);
+    for (int r = 0; r < RW; ++r) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < RW; ++r)
+        if (n0 + r < p.N) p.y[static_cast<size_t>(m) * p.N + n0 + r] = f32_to_bf16(scale * acc[r]);
+    }
   }
 }
 
