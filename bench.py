@@ -151,8 +151,11 @@ def workload(name):
             x = synth.normal_bf16((M, K), seed=8110 + bits)
             s = synth.bf16_bits(torch.tensor([0.0123]))
             nb = N * K * bits // 8 + 2 + 2 * M * K + 2 * M * N
+            # ALU bound: per value the state's inst3 multiply-add, its mask
+            # and XOR (one 3-input logic op), the binary16 addition of the two
+            # halves, the conversion to fp32 and the fused multiply-add
             L.append(Launch(f"trellis_b{bits}", "trellis", nb, M=M, N=N, K=K, bits=bits, gs=0,
-                            x=x, w=w, s=s))
+                            x=x, w=w, s=s, alu_ops=TRELLIS_OPS_PER_VALUE * M * N * K))
         cfg = {"workload": "trellis-mode decode GEMV", "M": M, "K": K, "N": N, "bits": [2, 4]}
     elif name == "quantize":
         # the producer side of the format on the decode weight shape: one
@@ -400,6 +403,22 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# Operations per trellis value (see the trellis workload) and the ALU peak:
+# 148 SMs x 128 FP32 lanes x the maximum SM clock (operations per second).
+TRELLIS_OPS_PER_VALUE = 5
+ALU_LANES = 148 * 128
+
+
+def alu_peak():
+    """Lane operations per second at the maximum SM clock, in Gop/s."""
+    mhz = 1965.0
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    return ALU_LANES * mhz * 1e6 / 1e9, "derived (148 SMs x 128 lanes x max SM clock)"
+
+
 def measured_tensor_peak():
     """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -639,6 +658,16 @@ def _roofline(l, ms, peak, peak_kind, tpeak, tpeak_kind, basis, traffic):
     """The bound of launch l: HBM bytes, or tensor FLOPs where the launch
     carries them and their time at the measured tensor peak is the longer."""
     t_mem = l.nbytes / (peak * 1e9)
+    ops = getattr(l, "alu_ops", None)
+    if ops:
+        apeak, akind = alu_peak()
+        if ops / (apeak * 1e9) > t_mem:
+            ach = ops / (ms * 1e-3) / 1e9
+            return {"bound": "alu", "kernel": l.label, "achieved": round(ach, 1),
+                    "peak": round(apeak, 1), "unit": "Gop/s", "frac": round(ach / apeak, 4),
+                    "peak_kind": akind, "timing": basis, "traffic": traffic,
+                    "algorithmic_ops_per_launch": ops,
+                    "algorithmic_bytes_per_launch": l.nbytes}
     flops = getattr(l, "flops", None)
     if flops and flops / (tpeak * 1e12) > t_mem:
         ach = flops / (ms * 1e-3) / 1e12

@@ -238,3 +238,15 @@ def test_prefill_launches_carry_their_flops():
     for l in launches:
         assert l.flops == 2 * l.M * l.N * l.K
         assert l.nbytes == _arrays_bytes(l.w, l.s, l.b, l.x) + 2 * l.M * l.N
+
+
+def test_trellis_roofline_is_alu_bound():
+    # 5 operations per value over 58.7M values at the derived ALU peak take
+    # longer than the launch's 29 MB at the HBM peak
+    launches, _ = bench.workload("trellis")
+    for l in launches:
+        assert l.alu_ops == bench.TRELLIS_OPS_PER_VALUE * l.M * l.N * l.K
+        r = bench._roofline(l, 0.036, 6537.0, "measured", 1627.7, "measured", "b", None)
+        assert r["bound"] == "alu" and r["unit"] == "Gop/s"
+        assert abs(r["peak"] - bench.alu_peak()[0]) < 0.1
+        assert abs(r["achieved"] * 0.036e-3 * 1e9 - l.alu_ops) < 1e-3 * l.alu_ops
