@@ -189,8 +189,30 @@ __device__ __forceinline__ uint32_t quantize_code(float v, float bias, float sca
   return static_cast<uint32_t>(fminf(code, n_bins));
 }
 
-// One work item: 32 chunks (one warp, lane = chunk).  Computes the group
-// parameters with xor butterflies over the group's lanes, stores the group's
+// The affine map of one group from its range [lo, hi] (lo taken from the
+// largest finite bf16 down, hi from 0 up, as the page's affine_quantize
+// starts them), in binary32 with IEEE divisions:
+//   * the code step has magnitude max((hi - lo) / n_bins, 1e-7);
+//   * the anchor is the endpoint of larger magnitude (hi on a tie); the step
+//     takes the anchor's sign when the anchor is lo, the opposite sign when
+//     it is hi, so codes grow away from the anchor into the range;
+//   * the anchor's position on the code grid, j = round(anchor / step)
+//     (halves away from zero), refines the step to anchor / j, and the
+//     anchor becomes the offset -- unless j = 0, when the step stays and the
+//     offset is 0.
+// Returns the step (the stored scale) and the offset (the stored bias).
+__device__ __forceinline__ float2 group_step_offset(float lo, float hi, float n_bins) {
+  const float magnitude = fmaxf(__fdiv_rn(__fsub_rn(hi, lo), n_bins), 1e-7f);
+  const bool anchor_is_lo = fabsf(lo) > fabsf(hi);
+  const float anchor = anchor_is_lo ? lo : hi;
+  const float step = anchor_is_lo ? magnitude : -magnitude;
+  const float j = roundf(__fdiv_rn(anchor, step));
+  if (j == 0.0f) return make_float2(step, 0.0f);
+  return make_float2(__fdiv_rn(anchor, j), anchor);
+}
+
+// One work item: 32 chunks (one warp, lane = chunk).  Finds the group's
+// range with xor butterflies over the group's lanes, stores the group's
 // scale and bias from its first lane and the lane's packed codes.
 template <int BITS, int GS>
 __device__ __forceinline__ void quantize_item(const uint4 raw, long long c, bool live, int lane,
@@ -199,8 +221,7 @@ __device__ __forceinline__ void quantize_item(const uint4 raw, long long c, bool
                                               uint16_t *__restrict__ biases) {
   constexpr int kLanes = GS / 8;  // lanes per group
   const float n_bins = static_cast<float>((1 << BITS) - 1);
-  const float eps = 1e-7f;
-  const float start_min = bf16_bits_to_float(0x7f7fu);  // largest finite bf16
+  const float start_lo = bf16_bits_to_float(0x7f7fu);  // largest finite bf16
   const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
   float v[8];
 #pragma unroll
@@ -208,25 +229,19 @@ __device__ __forceinline__ void quantize_item(const uint4 raw, long long c, bool
     v[2 * i] = __uint_as_float(pr[i] << 16);
     v[2 * i + 1] = __uint_as_float(pr[i] & 0xffff0000u);
   }
-  float w_min = start_min, w_max = 0.0f;
+  float lo = start_lo, hi = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    w_min = fminf(w_min, v[i]);
-    w_max = fmaxf(w_max, v[i]);
+    lo = fminf(lo, v[i]);
+    hi = fmaxf(hi, v[i]);
   }
 #pragma unroll
   for (int o = 1; o < kLanes; o <<= 1) {
-    w_min = fminf(w_min, __shfl_xor_sync(0xffffffffu, w_min, o));
-    w_max = fmaxf(w_max, __shfl_xor_sync(0xffffffffu, w_max, o));
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
-  float scale = fmaxf(__fdiv_rn(__fsub_rn(w_max, w_min), n_bins), eps);
-  const bool side = fabsf(w_min) > fabsf(w_max);
-  scale = side ? scale : -scale;
-  const float edge = side ? w_min : w_max;
-  const float q0 = roundf(__fdiv_rn(edge, scale));
-  const bool at_zero = q0 == 0.0f;
-  scale = at_zero ? scale : __fdiv_rn(edge, q0);
-  const float bias = at_zero ? 0.0f : edge;
+  const float2 so = group_step_offset(lo, hi, n_bins);
+  const float scale = so.x, bias = so.y;
   if (live && (lane % kLanes) == 0) {
     const long long g = c / kLanes;
     scales[g] = __bfloat16_as_ushort(__float2bfloat16_rn(scale));
