@@ -849,6 +849,10 @@ int launch_qvm_t(const qmvk::QvmParams &p, cudaStream_t stream) {
 // (N / gs) % 8 == 0); other shapes take qvm_kernel.
 // Dynamic shared memory of the staged qvm: the CTA's activations (fp32),
 // 128 bytes of alignment slack, the stages.
+// Rows of a column block are split between the CTAs of one cluster: 16 where
+// the device allows clusters that large (twice the CTAs in flight), else 8.
+constexpr int kQvtClusterBig = 16;
+
 int qvm_tma_smem(int K, int bits, uint32_t *ring_off, uint32_t *stage_bytes) {
   const int xrows = (K + qmvk::kQvmCluster - 1) / qmvk::kQvmCluster + 1;
   *ring_off = static_cast<uint32_t>((4LL * xrows + 127) / 128 * 128);
@@ -894,16 +898,44 @@ int launch_qvm_tma_t(const qmvk::QvmParams &q, DeviceInfo *dev, cudaStream_t str
     granted[d] = smem;
   }
   const int nblk = (q.N + qmvk::kQvmCols - 1) / qmvk::kQvmCols;
+  // the larger cluster where the device can hold one at this size (asked
+  // once per device), else the portable size
+  static int big_ok[kMaxDevices] = {};  // 0 unknown, 1 yes, 2 no
+  if (!big_ok[d]) {
+    big_ok[d] = 2;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t oc = {};
+      oc.gridDim = dim3(nblk, kQvtClusterBig, 1);
+      oc.blockDim = dim3((qmvk::kQvtWarps + 1) * 32);
+      oc.dynamicSmemBytes = static_cast<size_t>(smem);
+      cudaLaunchAttribute ca[1];
+      ca[0].id = cudaLaunchAttributeClusterDimension;
+      ca[0].val.clusterDim.x = 1;
+      ca[0].val.clusterDim.y = kQvtClusterBig;
+      ca[0].val.clusterDim.z = 1;
+      oc.attrs = ca;
+      oc.numAttrs = 1;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, kern, &oc) == cudaSuccess && nc >= 1) big_ok[d] = 1;
+    }
+    cudaGetLastError();  // a refused size leaves no error behind
+  }
+  const int ncl = big_ok[d] == 1 ? kQvtClusterBig : qmvk::kQvmCluster;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nblk, qmvk::kQvmCluster, q.M);
+  cfg.gridDim = dim3(nblk, ncl, q.M);
   cfg.blockDim = dim3((qmvk::kQvtWarps + 1) * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = ncl;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tw, ts, tb, p);
   if (le != cudaSuccess) {
     cudaGetLastError();  // clear it

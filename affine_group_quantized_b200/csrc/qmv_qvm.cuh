@@ -199,8 +199,9 @@ struct QvtParams {
   uint32_t ring_off;      // smem offset of the stages (rounded up to 128 in the kernel)
 };
 
+// The cluster (its size set at launch: gridDim.y CTAs share a column block)
 template <int BITS>
-__global__ void __cluster_dims__(1, kQvmCluster, 1) __launch_bounds__((kQvtWarps + 1) * 32, 1)
+__global__ void __launch_bounds__((kQvtWarps + 1) * 32, 1)
     qvm_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                    const __grid_constant__ CUtensorMap tm_b, const QvtParams p) {
   namespace cg = cooperative_groups;
@@ -216,8 +217,9 @@ __global__ void __cluster_dims__(1, kQvmCluster, 1) __launch_bounds__((kQvtWarps
   const int nb = blockIdx.x, rank = blockIdx.y, m = blockIdx.z;
   const int c = nb * 32 + lane;               // this lane's chunk of 8 columns
   const bool live = 8 * c < p.N;
-  const int k0 = static_cast<int>(static_cast<long long>(p.K) * rank / kQvmCluster);
-  const int k1 = static_cast<int>(static_cast<long long>(p.K) * (rank + 1) / kQvmCluster);
+  const int ncl = static_cast<int>(gridDim.y);  // CTAs of the cluster (row split)
+  const int k0 = static_cast<int>(static_cast<long long>(p.K) * rank / ncl);
+  const int k1 = static_cast<int>(static_cast<long long>(p.K) * (rank + 1) / ncl);
   const int nstg = (k1 - k0 + kQvtRows - 1) / kQvtRows;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t ring = (sbase + p.ring_off + 127u) & ~127u;  // 128 bytes of slack
@@ -319,7 +321,7 @@ __global__ void __cluster_dims__(1, kQvmCluster, 1) __launch_bounds__((kQvtWarps
     for (int col = threadIdx.x; col < kQvmCols; col += blockDim.x) {
       const int n = nb * kQvmCols + col;
       float sum = 0.f;
-      for (int r = 0; r < kQvmCluster; ++r) sum += cluster.map_shared_rank(part, r)[col];
+      for (int r = 0; r < ncl; ++r) sum += cluster.map_shared_rank(part, r)[col];
       if (n < p.N) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16(sum);
     }
   }
