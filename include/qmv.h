@@ -127,8 +127,9 @@ int qmv_noalloc(const void *x, const uint32_t *w, const void *scales,
  *   y       bf16 [M, N]  (written; must not overlap the inputs)
  *   y[m][n] = sum_k x[m][k] * (scale[k][n/gs] * q[k][n] + bias[k][n/gs])
  * N a positive multiple of group_size, K >= 1, 1 <= M <= 65535.  The rows
- * are split between the CTAs of a thread-block cluster whose partial sums
- * are added in a fixed order (deterministic results, no scratch memory).
+ * are split between the CTAs of a thread-block cluster (8, or 16 where the
+ * device allows) whose partial sums are added in a fixed order
+ * (deterministic results, no scratch memory).
  */
 int qvm(const void *x, const uint32_t *w, const void *scales, const void *biases, void *y,
         int M, int K, int N, int bits, int group_size, void *stream);
