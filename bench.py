@@ -213,33 +213,37 @@ def _outputs(l):
 
 
 class _Packed:
-    """One device buffer (and one pinned host buffer) holding several arrays
-    back to back at 16-byte aligned offsets, each reachable as a typed view:
-    a step's host copies are then one transfer each way."""
+    """Device buffers (and pinned host buffers) holding several arrays back to
+    back at 16-byte aligned offsets, each reachable as a typed view: a step's
+    host copies are then one transfer each way.  `slots` independent copies
+    (one per step of a weight rotation) let the copies of one step overlap
+    the launches of another."""
 
-    def __init__(self, specs, torch):
+    def __init__(self, specs, torch, slots=1):
         self.offsets, off = [], 0
         for _, shape, dt in specs:
             nb = int(np.prod(shape)) * np.dtype(dt).itemsize
             self.offsets.append((off, nb, shape, dt))
             off += (nb + 15) // 16 * 16
         self.nbytes = max(off, 16)
-        self.dev = torch.empty(self.nbytes, dtype=torch.uint8, device="cuda")
-        self.host = torch.empty(self.nbytes, dtype=torch.uint8).pin_memory()
+        self.slots = slots
+        self.dev = torch.empty((slots, self.nbytes), dtype=torch.uint8, device="cuda")
+        self.host = torch.empty((slots, self.nbytes), dtype=torch.uint8).pin_memory()
         self.names = [n for n, _, _ in specs]
         self.torch = torch
 
-    def view(self, i, buf=None):
+    def view(self, i, slot=0):
         torch = self.torch
         off, nb, shape, dt = self.offsets[i]
-        t = (self.dev if buf is None else buf)[off:off + nb]
+        t = self.dev[slot % self.slots][off:off + nb]
         td = {np.uint16: torch.bfloat16, np.uint32: torch.int32, np.int32: torch.int32}[dt]
         return t.view(td).view(shape)
 
     def fill_host(self, arrays):
         h = self.host.numpy()
-        for (off, nb, _, _), a in zip(self.offsets, arrays):
-            h[off:off + nb] = np.frombuffer(np.ascontiguousarray(a).tobytes(), np.uint8)
+        for slot in range(self.slots):
+            for (off, nb, _, _), a in zip(self.offsets, arrays):
+                h[slot, off:off + nb] = np.frombuffer(np.ascontiguousarray(a).tobytes(), np.uint8)
 
 
 class DeviceWorkload:
@@ -247,7 +251,7 @@ class DeviceWorkload:
     `copies[i]` copies per launch i; each launch's per-step inputs and its
     outputs are views into one packed input and one packed output buffer."""
 
-    def __init__(self, launches, copies, torch):
+    def __init__(self, launches, copies, torch, slots=1):
         import affine_group_quantized_b200 as agq
         self.agq, self.torch, self.launches = agq, torch, launches
         self.weights = []
@@ -267,8 +271,9 @@ class DeviceWorkload:
                 idx[k] = len(out_specs)
                 out_specs.append((k, shape, dt))
             self.out_idx.append(idx)
-        self.inp = _Packed(in_specs, torch)
-        self.out = _Packed(out_specs, torch)
+        self.slots = slots
+        self.inp = _Packed(in_specs, torch, self.slots)
+        self.out = _Packed(out_specs, torch, self.slots)
         arrays = [np.ascontiguousarray(getattr(l, k)) for l in launches for k in _INPUTS[l.kind]]
         self.inp.fill_host(arrays)
         self.inp.dev.copy_(self.inp.host)
@@ -280,8 +285,8 @@ class DeviceWorkload:
         quantizer reads the matrix just copied in from the host."""
         l, agq = self.launches[i], self.agq
         c = self.weights[i][k % len(self.weights[i])]
-        I = {n: self.inp.view(j) for n, j in self.in_idx[i].items()}
-        O = {n: self.out.view(j) for n, j in self.out_idx[i].items()}
+        I = {n: self.inp.view(j, k) for n, j in self.in_idx[i].items()}
+        O = {n: self.out.view(j, k) for n, j in self.out_idx[i].items()}
         if l.kind == "qmv":
             agq.qmv(I["x"], c["w"], c["s"], c["b"], O["y"], l.M, l.N, l.K, l.bits, l.gs)
         elif l.kind == "trellis":
@@ -310,9 +315,43 @@ class DeviceWorkload:
     def e2e_step(self, k):
         """One step as a user runs it: inputs in from pinned host memory, the
         launches, the outputs back to pinned host memory."""
-        self.inp.dev.copy_(self.inp.host, non_blocking=True)
+        slot = k % self.slots
+        self.inp.dev[slot].copy_(self.inp.host[slot], non_blocking=True)
         self.step(k, e2e=True)
-        self.out.host.copy_(self.out.dev, non_blocking=True)
+        self.out.host[slot].copy_(self.out.dev[slot], non_blocking=True)
+
+    def e2e_rotation(self, side):
+        """The steps of one weight rotation as a pipelined serving loop runs
+        them: every step's inputs go in from pinned host memory and its
+        outputs come back, one copy each way per step, on a second stream;
+        step k's launches wait for its own inputs only, and its outputs leave
+        once its launches are done, while later steps compute."""
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        landed = []
+        with torch.cuda.stream(side):
+            for k in range(self.slots):
+                self.inp.dev[k].copy_(self.inp.host[k], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(side)
+                landed.append(e)
+        done = []
+        for k in range(self.slots):
+            main.wait_event(landed[k])
+            self.step(k, e2e=True)
+            e = torch.cuda.Event()
+            e.record(main)
+            done.append(e)
+        with torch.cuda.stream(side):
+            for k in range(self.slots):
+                side.wait_event(done[k])
+                self.out.host[k].copy_(self.out.dev[k], non_blocking=True)
+            join = torch.cuda.Event()
+            join.record(side)
+        main.wait_event(join)
 
 
 class ClockSampler:
@@ -513,7 +552,7 @@ def measure_workload(name, args, torch, world, with_cpu):
     flush = step_bytes < 64 * 2**20
     copies = 1 if flush else max(2, -(-2 * L2_BYTES // step_bytes) + 1)
     per = [copies if flush else max(copies, -(-2 * L2_BYTES // l.nbytes) + 1) for l in launches]
-    dw = DeviceWorkload(launches, per, torch)
+    dw = DeviceWorkload(launches, per, torch, slots=copies)
     scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
 
     def step(k):
@@ -576,22 +615,30 @@ def measure_workload(name, args, torch, world, with_cpu):
 
     # End to end through the public API: per step, the step's inputs in from
     # pinned host memory (one copy), the launches, the outputs back to pinned
-    # host memory (one copy); one CUDA graph per step.
+    # host memory (one copy).  A weight rotation's steps run as one CUDA
+    # graph in which the copies go over a second stream and overlap the
+    # other steps' launches (a pipelined serving loop); the remaining steps
+    # run one graph each.
+    side = torch.cuda.Stream()
     for k in range(copies):
         dw.e2e_step(k)
     torch.cuda.synchronize()
+    erot = _graph(torch, lambda: dw.e2e_rotation(side))
     egraphs = [_graph(torch, lambda c=c: dw.e2e_step(c)) for c in range(copies)]
+    erot.replay()
     for g in egraphs:
         g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for k in range(K):
-        egraphs[k % copies].replay()
+    for _ in range(K // copies):
+        erot.replay()
+    for k in range(K % copies):
+        egraphs[k].replay()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
-    del egraphs
+    del egraphs, erot
 
     peak, peak_kind = measured_peaks()
     out_launch = {}
@@ -640,9 +687,12 @@ def measure_workload(name, args, torch, world, with_cpu):
         "e2e": {"value": round(job_gbs(world, step_bytes, K, e2e_ms), 1),
                 "unit": UNIT, "h2d_bytes_per_step": dw.h2d_bytes,
                 "d2h_bytes_per_step": dw.d2h_bytes,
-                "note": "weights resident in HBM; each step's inputs copied in (one "
-                        "copy) and outputs copied out (one copy); each step replayed "
-                        "as one CUDA graph"},
+                "note": "weights resident in HBM; each step's inputs copied in from "
+                        "pinned host memory (one copy) and outputs copied out (one "
+                        "copy); the copies of a weight rotation's steps run on a second "
+                        "stream and overlap the other steps' launches (a step's "
+                        "launches wait for its own inputs, its outputs leave when its "
+                        "launches are done); each rotation replayed as one CUDA graph"},
         "gpu_launches": K * len(launches),
         "clocks": sampler.summary(),
     }
